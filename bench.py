@@ -1,0 +1,435 @@
+#!/usr/bin/env python
+"""Benchmark of the block-sparse prefill hot path on B200.
+
+One step = one layer of the workload through the whole path: block pattern
+discovery + index compaction (fused launch) and block-sparse attention, on
+inputs already resident in HBM. Default workload: 128K-token prefill with
+Qwen3-30B-A3B-like attention (Hq=32, Hkv=4, d=128, block 128, alpha 0.1,
+sink 256, window 512, ~5% of causal blocks kept), bf16.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                       [--workload NAME] [--dtype bf16|e4m3]
+Multi-GPU (weak scaling, every rank runs its own layer, no data-path collective):
+  python -m torch.distributed.run --nproc-per-node N --master-addr 127.0.0.1 bench.py --gpus N
+
+Prints one JSON line (rank 0). value = dense-equivalent TFLOP/s of the step
+(4*d*Hq*sum L(L+1)/2 per layer) over all ranks; ms_per_step = ms per layer.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from block_sparse_long_blocks_b200 import workloads as wl  # noqa: E402
+
+METRIC = "sparse prefill attn ms/layer & dense-equiv TFLOPS @128K; % of TC peak"
+UNIT = "TFLOPS (dense-equivalent)"
+FP8_OVER_BF16 = 2.0  # nominal dense fp8 / bf16 tensor-core ratio (4.5 / 2.25 PFLOP/s)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    fp8=float(d["fp8_tflops"]) if "fp8_tflops" in d else None, source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, fp8=None, source="fallback")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            props = torch.cuda.get_device_properties(device_index)
+            self.sel = "GPU-" + str(props.uuid)
+        except Exception:
+            self.sel = str(device_index)
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- oracle baseline
+def oracle_sample(w: wl.Workload, inp: wl.Inputs, budget_s: float, max_rows: int, seed: int = 0):
+    """Time the CPU oracle on a bounded sample of (KV group, query block) rows of
+    the first request and extrapolate to the whole layer by work counts."""
+    import oracle
+    from tests import _helpers as H
+
+    q, k, v = H.request_views(inp)[0]
+    B, G = w.block, w.group
+    scale = oracle.default_scale(w.head_dim)
+    Sb, Wb = oracle.forced_blocks(w.sink_tokens, w.window_tokens, B)
+    L = q.shape[0]
+    N = -(-L // B)
+    t0 = time.perf_counter()
+    kbar = H.pooled_f64(k, B, inp.k_scale)  # all key blocks (every row needs them)
+    t_kpool = time.perf_counter() - t0
+    Qv, Kv, Vv = H.Lazy64(q, inp.q_scale), H.Lazy64(k, inp.k_scale), H.Lazy64(v, inp.v_scale)
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(N * w.hkv)
+    t_disc = t_attn = 0.0
+    rows = 0
+    score_work = 0        # sum over sampled rows of (i + 1)
+    visits = 0
+    for u in order[:max_rows]:
+        g, i = int(u % w.hkv), int(u // w.hkv)
+        t1 = time.perf_counter()
+        lo, hi = i * B, min((i + 1) * B, L)
+        qs = None if inp.q_scale is None else inp.q_scale[g * G:(g + 1) * G]
+        qbar_i = oracle.pool_blocks(H.f64(q[lo:hi, g * G:(g + 1) * G], qs), B)[0]
+        lst = oracle.discover_row(qbar_i, kbar[:, g], i, scale, w.alpha, Sb, Wb)
+        t2 = time.perf_counter()
+        oracle.attention_rows(Qv, Kv, Vv, g, i, lst, B, scale)
+        t3 = time.perf_counter()
+        t_disc += t2 - t1
+        t_attn += t3 - t2
+        rows += 1
+        score_work += i + 1
+        visits += len(lst)
+        if t_kpool + t_disc + t_attn > budget_s:
+            break
+    return dict(t_kpool=t_kpool, t_disc=t_disc, t_attn=t_attn, rows=rows, score_work=score_work,
+                visits=visits, N=N, wall=t_kpool + t_disc + t_attn)
+
+
+def extrapolate(s: dict, w: wl.Workload, total_visits: int) -> float:
+    """Seconds the oracle would take for the whole layer, from a sample's rates."""
+    N, rows = s["N"], max(1, s["rows"])
+    total_rows = N * w.hkv
+    total_score = w.hkv * N * (N + 1) / 2
+    # discovery per row = q-block pooling (constant) + scoring (proportional to i + 1)
+    disc = s["t_disc"] * 0.5 * (total_rows / rows + total_score / max(1, s["score_work"]))
+    attn = s["t_attn"] * total_visits / max(1, s["visits"])
+    return s["t_kpool"] + disc + attn
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="qwen30b_128k")
+    ap.add_argument("--dtype", default="bf16", choices=["bf16", "e4m3"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-fp8-extra", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "native":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist_mod
+        dist = dist_mod
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+
+    w = wl.workloads()[args.workload]
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, w, world)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+    line = run_native(args, w, world, rank, local, dist)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args, w, world):
+    inp = wl.make_inputs(w)
+    if args.dtype == "e4m3":
+        inp = wl.to_fp8(inp)
+    # the oracle's own lists give the visited-block count used for extrapolation
+    from tests import _helpers as H
+    orc = H.oracle_discovery(w, inp)
+    total_visits = int(sum(int(o["cnt"].sum()) for o in orc))
+    times = []
+    per_step_budget = max(2.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    last = None
+    for s in range(args.warmup + args.steps):
+        smp = oracle_sample(w, inp, per_step_budget, max_rows=64, seed=s)
+        if s >= args.warmup:
+            times.append(extrapolate(smp, w, total_visits))
+        last = smp
+    t = statistics.mean(times)
+    flops = w.dense_equiv_flops()
+    val = flops / t / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "seq_len": w.seqlens[0], "hq": w.hq, "hkv": w.hkv, "block": w.block,
+                       "alpha": w.alpha, "input_dtype": args.dtype},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+                             "sample": f"per step {last['rows']} (KV group, query block) rows of the layer "
+                                       f"(discovery + attention) plus full key pooling, extrapolated by work "
+                                       f"counts to all {last['N'] * w.hkv} rows / {total_visits} visited blocks"},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_native(args, w, world, rank, local, dist):
+    from block_sparse_long_blocks_b200 import binding as fb
+
+    fb.load()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pk = peaks()
+    inp_host = wl.make_inputs(w)
+    fp8 = args.dtype == "e4m3"
+    if fp8:
+        inp_host = wl.to_fp8(inp_host)
+
+    def setup(inp):
+        cfg = fb.config_for(w, inp)
+        t = lambda x: None if x is None else x.to(dev).contiguous()  # noqa: E731
+        paged = inp.page_table is not None
+        d = dict(q=t(inp.q), k=t(inp.k if not paged else inp.k_pool), v=t(inp.v if not paged else inp.v_pool),
+                 cu=t(inp.cu_seqlens), table=t(inp.page_table), qs=t(inp.q_scale), ks=t(inp.k_scale),
+                 vs=t(inp.v_scale), paged=paged, cfg=cfg)
+        d["p"] = fb.make_params(cfg, d["qs"], d["ks"], d["vs"], d["cu"], d["table"])
+        d["bufs"] = fb.Buffers(d["p"], device=dev, o_shape=tuple(inp.q.shape))
+        return d
+
+    D = setup(inp_host)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        fb.fp_discover_compact(D["p"], D["q"], D["k"], None, D["bufs"].idx, D["bufs"].cnt, D["bufs"].workspace)
+        if ev is not None:
+            ev[1].record(stream)
+        if D["paged"]:
+            fb.fp_paged_sparse_prefill(D["p"], D["q"], D["k"], D["v"], D["bufs"].idx, D["bufs"].cnt, D["bufs"].o)
+        else:
+            fb.fp_sparse_prefill(D["p"], D["q"], D["k"], D["v"], D["bufs"].idx, D["bufs"].cnt, D["bufs"].o)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = fb.fp_get_device_status()
+    if status:
+        raise RuntimeError(f"device status {status:#x} after warm-up")
+
+    # timed region (inputs > L2: Q alone is 1 GiB, so no flush between steps)
+    clocks = ClockSampler(local)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    start.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if dist is not None:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    disc_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    if dist is not None:
+        t = torch.tensor([ms, disc_ms, attn_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, disc_ms, attn_ms = t.tolist()
+    ms_step = ms / args.steps
+
+    # work counts from the lists of the last step
+    cfg = D["cfg"]
+    cnt = D["bufs"].cnt.long()
+    visits = int(cnt.sum().item())
+    B, d, G = w.block, w.head_dim, w.group
+    visited_flops = visits * 4.0 * B * B * d * G
+    dense = w.dense_equiv_flops()
+    causal_pairs = w.hkv * sum((-(-L // B)) * ((-(-L // B)) + 1) // 2 for L in w.seqlens)
+    es = 1 if fp8 else 2
+    qk_bytes = (inp_host.q.numel() + (inp_host.k.numel() if inp_host.k is not None else inp_host.k_pool.numel())) * es
+    disc_bytes = qk_bytes + 4 * visits + 4 * cnt.numel()
+    peak_tc = (pk["fp8"] if (fp8 and pk["fp8"]) else pk["bf16"] * (FP8_OVER_BF16 if fp8 else 1.0))
+    achieved = visited_flops / (attn_ms * 1e-3) / 1e12
+    value = world * dense / (ms_step * 1e-3) / 1e12
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": args.dtype, "data": "synthetic (seeded Gaussian Q/K/V with heavy key "
+            "blocks and slash diagonals; no model weights)",
+            "config": {"workload": w.name, "seq_len": w.seqlens[0] if len(w.seqlens) == 1 else list(w.seqlens),
+                       "global_batch": world * len(w.seqlens), "hq": w.hq, "hkv": w.hkv, "head_dim": d,
+                       "block": B, "alpha": w.alpha, "sink_tokens": w.sink_tokens,
+                       "window_tokens": w.window_tokens, "parallelism": f"replicas{world} (one layer per rank)",
+                       "l2": "inputs larger than L2 (Q alone 1 GiB); no flush",
+                       "density": visits / causal_pairs},
+            "ms_per_layer": ms_step, "discover_compact_ms": disc_ms, "attention_ms": attn_ms,
+            "visited_tile_tflops": achieved,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tc, "unit": "TFLOP/s",
+                         "frac": achieved / peak_tc, "traffic": None,
+                         "kernel": "sparse_attention_kernel",
+                         "peak_source": f"{pk['source']} bf16 burst" + (" x2 (nominal fp8/bf16)" if fp8 else "")},
+            "discovery_roofline": {"bound": "hbm", "achieved": disc_bytes / (disc_ms * 1e-3) / 1e9,
+                                   "peak": pk["hbm"], "unit": "GB/s",
+                                   "frac": disc_bytes / (disc_ms * 1e-3) / 1e9 / pk["hbm"],
+                                   "algorithmic_bytes": disc_bytes},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clk}
+
+    # end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    if not args.no_e2e:
+        line["e2e"] = e2e(args, D, inp_host, dev, stream, dense, world, dist)
+    if fp8 is False and not args.no_fp8_extra:
+        line["fp8"] = fp8_extra(args, w, inp_host, dev, stream, pk, setup, dist)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        smp = oracle_sample(w, inp_host, args.cpu_budget, max_rows=10_000)
+        t = extrapolate(smp, w, visits)
+        line["cpu_baseline"] = {"value": dense / t / 1e12, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+                                "sample": f"{smp['rows']} (KV group, query block) rows of the layer (discovery + "
+                                          f"attention, {smp['wall']:.1f} s) plus full key pooling, extrapolated by "
+                                          f"work counts to {smp['N'] * w.hkv} rows / {visits} visited blocks",
+                                "extrapolated_s_per_layer": t}
+    return line
+
+
+def e2e(args, D, inp_host, dev, stream, dense, world, dist):
+    from block_sparse_long_blocks_b200 import binding as fb
+    paged = D["paged"]
+    hq = inp_host.q.pin_memory()
+    hk = (inp_host.k if not paged else inp_host.k_pool).pin_memory()
+    hv = (inp_host.v if not paged else inp_host.v_pool).pin_memory()
+    ho = torch.empty(tuple(inp_host.q.shape), dtype=torch.bfloat16).pin_memory()
+    h2d = hq.numel() * hq.element_size() + hk.numel() * hk.element_size() + hv.numel() * hv.element_size()
+    d2h = ho.numel() * ho.element_size()
+    steps = max(3, min(args.steps, 5))
+
+    def one():
+        D["q"].copy_(hq, non_blocking=True)
+        D["k"].copy_(hk, non_blocking=True)
+        D["v"].copy_(hv, non_blocking=True)
+        fb.fp_discover_compact(D["p"], D["q"], D["k"], None, D["bufs"].idx, D["bufs"].cnt, D["bufs"].workspace)
+        if paged:
+            fb.fp_paged_sparse_prefill(D["p"], D["q"], D["k"], D["v"], D["bufs"].idx, D["bufs"].cnt, D["bufs"].o)
+        else:
+            fb.fp_sparse_prefill(D["p"], D["q"], D["k"], D["v"], D["bufs"].idx, D["bufs"].cnt, D["bufs"].o)
+        ho.copy_(D["bufs"].o, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+    return {"value": world * dense / (ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
+
+
+def fp8_extra(args, w, inp_host, dev, stream, pk, setup, dist):
+    """Same step with FP8-e4m3 inputs (per-head absmax scales): ms/layer and fractions."""
+    from block_sparse_long_blocks_b200 import binding as fb
+    inp8 = wl.to_fp8(inp_host)
+    D = setup(inp8)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    disc, attn, tot = [], [], []
+    for s in range(args.warmup + args.steps):
+        ev[0].record(stream)
+        fb.fp_discover_compact(D["p"], D["q"], D["k"], None, D["bufs"].idx, D["bufs"].cnt, D["bufs"].workspace)
+        ev[1].record(stream)
+        fb.fp_sparse_prefill(D["p"], D["q"], D["k"], D["v"], D["bufs"].idx, D["bufs"].cnt, D["bufs"].o)
+        ev[2].record(stream)
+        torch.cuda.synchronize()
+        if s >= args.warmup:
+            disc.append(ev[0].elapsed_time(ev[1]))
+            attn.append(ev[1].elapsed_time(ev[2]))
+            tot.append(ev[0].elapsed_time(ev[2]))
+    visits = int(D["bufs"].cnt.long().sum().item())
+    flops = visits * 4.0 * w.block * w.block * w.head_dim * w.group
+    a = statistics.mean(attn)
+    peak = pk["fp8"] if pk["fp8"] else pk["bf16"] * FP8_OVER_BF16
+    del D
+    return {"ms_per_layer": statistics.mean(tot), "discover_compact_ms": statistics.mean(disc), "attention_ms": a,
+            "dense_equiv_tflops": w.dense_equiv_flops() / (statistics.mean(tot) * 1e-3) / 1e12,
+            "visited_tile_tflops": flops / (a * 1e-3) / 1e12,
+            "frac_of_fp8_peak": flops / (a * 1e-3) / 1e12 / peak,
+            "fp8_peak": peak, "fp8_peak_source": "measured" if pk["fp8"] else "bf16 measured x2 (nominal ratio)"}
+
+
+if __name__ == "__main__":
+    main()

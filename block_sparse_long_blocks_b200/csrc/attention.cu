@@ -1,0 +1,634 @@
+// Block-sparse causal prefill attention over compacted KV-block lists, sm_100a.
+//
+// "FlashPrefill V2" abstract: the sparse operator uses PackGQA memory access,
+// warp specialisation and ping-pong pipelining, supports FP8, paged KV and
+// continuous batching. FlashPrefill summary, Method 3: the inner loop visits
+// only the listed blocks ("physical jumps").
+//
+// Work unit = (request r, KV group kvh, query block i, M-tile pair). PackGQA:
+// the rows of an M-tile are (token, head) pairs of one KV group, token-major
+// (row = t * G + h), Tm tokens x G heads with Tm the largest power of two such
+// that Tm * G <= 128, so every K/V tile a CTA loads serves all G heads. A CTA
+// owns two M-tiles (ping-pong) and walks row (r, kvh, i)'s list.
+//
+// Roles (320 threads, one persistent CTA per SM):
+//   warps 0-3  softmax warpgroup for M-tile 0 (one thread per row)
+//   warps 4-7  softmax warpgroup for M-tile 1
+//   warp 8     TMA producer: Q tiles, then K[idx[n]] and V[idx[n]] into rings
+//   warp 9     MMA issuer (one thread): S = Q K^T into TMEM, O += P V with P
+//              read from TMEM (aliasing S), accumulators in TMEM
+// Order of MMAs per visit n (ping-pong): PV0(n), S0(n+1), PV1(n), S1(n+1), so
+// one warpgroup's softmax overlaps the other tile's MMAs.
+// Softmax: online, base-2, with the running reference max raised only when the
+// tile max exceeds it by more than 8 (then O and l are rescaled in place).
+// Every wait is time-bounded; on expiry the CTA records FP_DEV_TIMEOUT, drains
+// its own copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include <mutex>
+
+#include "internal.cuh"
+#include "sm100.cuh"
+
+namespace fp {
+
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kSmemBudget = 200 * 1024;
+
+// 2^x with the MUFU.EX2 instruction (flush-to-zero, ~2 ulp); 2^-inf = +0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+struct AttnArgs {
+  Geometry g;
+  int Tm;       // tokens per M-tile
+  int rows;     // Tm * G rows in use per M-tile
+  int nPairs;   // M-tile pairs per query block
+  long long num_units;
+  long long T;  // rows of Q / O (R*L contiguous, total_tokens varlen)
+  float scale_log2;
+  const int32_t* idx;
+  const int32_t* cnt;
+  __nv_bfloat16* o;
+  float* lse;
+};
+
+template <bool FP8, int BLK>
+struct Cfg {
+  static constexpr int ES = FP8 ? 1 : 2;
+  static constexpr int DCH = FP8 ? 1 : 2;                 // 128-byte chunks along d
+  static constexpr int CH_ELEMS = 128 / DCH;              // elements per chunk
+  static constexpr int Q_TILE = DCH * 128 * 128;          // bytes per 128-row M-tile
+  static constexpr int KV_CHUNK = BLK * 128;              // bytes per d-chunk of a K/V tile
+  static constexpr int KV_TILE = DCH * KV_CHUNK;
+  static constexpr int STAGES_RAW = (kSmemBudget - 2 * Q_TILE) / (2 * KV_TILE);
+  static constexpr int STAGES = STAGES_RAW > 4 ? 4 : STAGES_RAW;
+  static constexpr int KSTEP_BYTES = 32;                  // K extent of one MMA (16 bf16 / 32 e4m3)
+  static constexpr int QK_STEPS = 128 * ES / KSTEP_BYTES; // 8 (bf16) / 4 (e4m3)
+  static constexpr int PV_KEYS = KSTEP_BYTES / ES;        // keys per PV MMA: 16 / 32
+  static constexpr int PV_STEPS = BLK / PV_KEYS;
+  static constexpr int NUM_BARS = 2 + 4 * STAGES + 6 + 1;
+  static constexpr int SMEM_USED = 1024 + 2 * Q_TILE + 2 * STAGES * KV_TILE + NUM_BARS * 8 + 16;
+  // more than half of the SM's shared memory: one CTA per SM, so the CTA's
+  // 512-column TMEM allocation never waits for a co-resident CTA
+  static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
+  static_assert(STAGES >= 2, "shared memory budget too small");
+};
+
+struct Unit {
+  int r, kvh, i, pair, off, len, count;
+  long long lbase, rowi;
+};
+
+__device__ __forceinline__ bool decode_unit(long long u, const AttnArgs& a, Unit& U) {
+  const Geometry& g = a.g;
+  const long long per_i = (long long)g.R * g.Hkv * a.nPairs;
+  U.i = g.Nmax - 1 - (int)(u / per_i);
+  long long rem = u % per_i;
+  U.pair = (int)(rem % a.nPairs);
+  rem /= a.nPairs;
+  U.kvh = (int)(rem % g.Hkv);
+  U.r = (int)(rem / g.Hkv);
+  request_span(g, U.r, U.off, U.len);
+  const int q0 = U.i * g.B;
+  if (q0 >= U.len) return false;
+  if (U.pair * 2 * a.Tm >= U.len - q0) return false;  // both M-tiles past the request's end
+  U.rowi = row_index(U.r, U.kvh, U.i, g.Hkv, g.Nmax);
+  U.lbase = list_row_base(U.r, U.kvh, U.i, g.Hkv, g.Nmax);
+  int c = __ldg(a.cnt + U.rowi);
+  if (c < 0 || c > U.i + 1) {
+    atomicOr(g.status, FP_DEV_BAD_LIST);
+    c = c < 0 ? 0 : U.i + 1;
+  }
+  U.count = c;
+  return true;
+}
+
+__device__ __forceinline__ int list_entry(const AttnArgs& a, const Unit& U, int n) {
+  int j = __ldg(a.idx + U.lbase + n);
+  if (j < 0 || j > U.i) {
+    atomicOr(a.g.status, FP_DEV_BAD_LIST);
+    j = U.i;
+  }
+  return j;
+}
+
+template <bool FP8, int BLK, bool PAGED>
+__device__ __forceinline__ void load_kv_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
+                                             const AttnArgs& a, const Unit& U, int j) {
+  using C = Cfg<FP8, BLK>;
+  const Geometry& g = a.g;
+  if constexpr (!PAGED) {
+#pragma unroll
+    for (int ch = 0; ch < C::DCH; ++ch)
+      tma_load_3d(dst + ch * C::KV_CHUNK, map, bar, ch * C::CH_ELEMS, U.kvh, U.off + j * BLK);
+  } else {
+    const int sub_rows = g.page_size < BLK ? g.page_size : BLK;
+    const int nsub = BLK / sub_rows;
+    for (int s = 0; s < nsub; ++s) {
+      const int tok = j * BLK + s * sub_rows;
+      int page = g.num_pages;  // out of range -> the copy fills zeros
+      if (tok < U.len) {
+        const int pg = __ldg(g.page_table + (long long)U.r * g.max_pages + (tok >> g.page_shift));
+        if (pg >= 0 && pg < g.num_pages) page = pg;
+        else atomicOr(g.status, FP_DEV_BAD_PAGE);
+      }
+      const int slot = tok & (g.page_size - 1);
+#pragma unroll
+      for (int ch = 0; ch < C::DCH; ++ch)
+        tma_load_4d(dst + ch * C::KV_CHUNK + s * sub_rows * 128, map, bar, ch * C::CH_ELEMS, U.kvh, slot, page);
+    }
+  }
+}
+
+template <bool FP8, int BLK, bool PAGED>
+__global__ void __maxnreg__(200)
+    sparse_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                            const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+  using C = Cfg<FP8, BLK>;
+  constexpr int S = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + 2 * C::Q_TILE;
+  uint8_t* sV = sK + S * C::KV_TILE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + S * C::KV_TILE);
+  uint64_t* q_full = bars;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;
+  uint64_t* k_empty = k_full + S;
+  uint64_t* v_full = k_empty + S;
+  uint64_t* v_empty = v_full + S;
+  uint64_t* s_full = v_empty + S;  // [2]
+  uint64_t* p_full = s_full + 2;   // [2]
+  uint64_t* o_full = p_full + 2;   // [2]
+  uint64_t* drain = o_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const Geometry& g = a.g;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(k_empty + s, 1);
+      mbar_init(v_full + s, 1);
+      mbar_init(v_empty + s, 1);
+    }
+    for (int m = 0; m < 2; ++m) {
+      mbar_init(s_full + m, 1);
+      mbar_init(p_full + m, 128);
+      mbar_init(o_full + m, 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  // Rows a.rows..127 of each M-tile are never written by the Q copies; keep them zero.
+  if (a.rows < 128) {
+    const int pad = (128 - a.rows) * 128;
+    for (int x = threadIdx.x * 16; x < 2 * C::DCH * pad; x += kThreads * 16) {
+      const int chunk = x / pad, o = x % pad;
+      *reinterpret_cast<uint4*>(sQ + chunk * 128 * 128 + a.rows * 128 + o) = make_uint4(0, 0, 0, 0);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      long long kt = 0, vt = 0, qn = 0;
+      const uint32_t q_bytes = 2u * C::DCH * a.rows * 128u;
+      bool ok = true;
+      for (long long u = blockIdx.x; u < a.num_units && ok; u += gridDim.x) {
+        Unit U;
+        if (!decode_unit(u, a, U) || U.count == 0) continue;
+        ok = mbar_wait(q_empty, (uint32_t)(qn & 1) ^ 1u, abort_flag, g.status, FP_DEV_TIMEOUT);
+        if (!ok) break;
+        mbar_arrive_expect_tx(q_full, q_bytes);
+        for (int mt = 0; mt < 2; ++mt) {
+          const int t = U.off + U.i * g.B + (U.pair * 2 + mt) * a.Tm;
+#pragma unroll
+          for (int ch = 0; ch < C::DCH; ++ch)
+            tma_load_3d(sQ + mt * C::Q_TILE + ch * 128 * 128, &tmQ, q_full, ch * C::CH_ELEMS, U.kvh * g.G, t);
+        }
+        ++qn;
+        for (int n = 0; n < U.count && ok; ++n) {
+          const int j = list_entry(a, U, n);
+          int st = (int)(kt % S);
+          ok = mbar_wait(k_empty + st, (uint32_t)((kt / S) & 1) ^ 1u, abort_flag, g.status, FP_DEV_TIMEOUT);
+          if (!ok) break;
+          mbar_arrive_expect_tx(k_full + st, C::KV_TILE);
+          load_kv_tile<FP8, BLK, PAGED>(sK + st * C::KV_TILE, &tmK, k_full + st, a, U, j);
+          ++kt;
+          st = (int)(vt % S);
+          ok = mbar_wait(v_empty + st, (uint32_t)((vt / S) & 1) ^ 1u, abort_flag, g.status, FP_DEV_TIMEOUT);
+          if (!ok) break;
+          mbar_arrive_expect_tx(v_full + st, C::KV_TILE);
+          load_kv_tile<FP8, BLK, PAGED>(sV + st * C::KV_TILE, &tmV, v_full + st, a, U, j);
+          ++vt;
+        }
+      }
+      if (*abort_flag) {
+        // let every copy this CTA issued land before the shared memory is released
+        int never = 0;
+        for (long long t = kt - 1; t >= 0 && t >= kt - S; --t)
+          mbar_wait(k_full + (int)(t % S), (uint32_t)((t / S) & 1), (volatile int*)&never, g.status, 0u);
+        for (long long t = vt - 1; t >= 0 && t >= vt - S; --t)
+          mbar_wait(v_full + (int)(t % S), (uint32_t)((t / S) & 1), (volatile int*)&never, g.status, 0u);
+        if (qn > 0) mbar_wait(q_full, (uint32_t)((qn - 1) & 1), (volatile int*)&never, g.status, 0u);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t fmt = FP8 ? 0u : 1u;
+      const uint32_t idesc_qk = instr_desc(fmt, 128, BLK, 0, 0);
+      const uint32_t idesc_pv = instr_desc(fmt, 128, 128, 0, 1);
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+      long long kt = 0, vt = 0, qn = 0;
+      long long pn[2] = {0, 0};
+      bool ok = true;
+
+      auto issue_qk = [&](int mt, int kst) {
+#pragma unroll
+        for (int ks = 0; ks < C::QK_STEPS; ++ks) {
+          const uint32_t boff = (uint32_t)(ks * C::KSTEP_BYTES);
+          const uint32_t ch = boff / 128, in = boff % 128;
+          const uint64_t ad = smem_desc_sw128(sQa + mt * C::Q_TILE + ch * 128 * 128 + in, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(sKa + kst * C::KV_TILE + ch * C::KV_CHUNK + in, 16, 1024);
+          if (FP8) umma_f8_ss(tmem + mt * 128, ad, bd, idesc_qk, ks > 0);
+          else umma_f16_ss(tmem + mt * 128, ad, bd, idesc_qk, ks > 0);
+        }
+      };
+      // P occupies the first columns of the M-tile's S region: bf16 pairs, or for
+      // e4m3 a high plane (BLK/4 columns) followed by the residual plane.
+      auto issue_pv = [&](int mt, int vst, bool acc) {
+#pragma unroll
+        for (int plane = 0; plane < (FP8 ? 2 : 1); ++plane) {
+#pragma unroll
+          for (int ks = 0; ks < C::PV_STEPS; ++ks) {
+            const uint32_t a_t = tmem + mt * 128 + plane * (BLK / 4) + ks * (C::PV_KEYS * C::ES / 4);
+            const uint64_t bd =
+                smem_desc_sw128(sVa + vst * C::KV_TILE + ks * C::PV_KEYS * 128, C::KV_CHUNK, 1024);
+            const uint32_t accum = (acc || ks > 0 || plane > 0) ? 1u : 0u;
+            if (FP8) umma_f8_ts(tmem + 256 + mt * 128, a_t, bd, idesc_pv, accum);
+            else umma_f16_ts(tmem + 256 + mt * 128, a_t, bd, idesc_pv, accum);
+          }
+        }
+      };
+
+      for (long long u = blockIdx.x; u < a.num_units && ok; u += gridDim.x) {
+        Unit U;
+        if (!decode_unit(u, a, U) || U.count == 0) continue;
+        ok = mbar_wait(q_full, (uint32_t)(qn & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
+        if (!ok) break;
+        ++qn;
+        int kst = (int)(kt % S);
+        ok = mbar_wait(k_full + kst, (uint32_t)((kt / S) & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
+        if (!ok) break;
+        tc_fence_after();
+        issue_qk(0, kst);
+        umma_commit(s_full + 0);
+        issue_qk(1, kst);
+        umma_commit(s_full + 1);
+        umma_commit(k_empty + kst);
+        ++kt;
+        if (U.count == 1) umma_commit(q_empty);
+        for (int n = 0; n < U.count; ++n) {
+          const int vst = (int)(vt % S);
+          ok = mbar_wait(v_full + vst, (uint32_t)((vt / S) & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
+          if (!ok) break;
+          ok = mbar_wait(p_full + 0, (uint32_t)(pn[0] & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
+          if (!ok) break;
+          ++pn[0];
+          tc_fence_after();
+          issue_pv(0, vst, n > 0);
+          const bool more = n + 1 < U.count;
+          if (more) {
+            kst = (int)(kt % S);
+            ok = mbar_wait(k_full + kst, (uint32_t)((kt / S) & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
+            if (!ok) break;
+            tc_fence_after();
+            issue_qk(0, kst);
+            umma_commit(s_full + 0);
+          } else {
+            umma_commit(o_full + 0);
+          }
+          ok = mbar_wait(p_full + 1, (uint32_t)(pn[1] & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
+          if (!ok) break;
+          ++pn[1];
+          tc_fence_after();
+          issue_pv(1, vst, n > 0);
+          umma_commit(v_empty + vst);
+          ++vt;
+          if (more) {
+            issue_qk(1, kst);
+            umma_commit(s_full + 1);
+            umma_commit(k_empty + kst);
+            ++kt;
+            if (n + 2 == U.count) umma_commit(q_empty);
+          } else {
+            umma_commit(o_full + 1);
+          }
+        }
+      }
+      // every MMA this thread issued has completed once `drain` flips
+      umma_commit(drain);
+      int never = 0;
+      mbar_wait(drain, 0u, (volatile int*)&never, g.status, FP_DEV_TIMEOUT);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax warpgroups
+    const int mt = warp >> 2;
+    const int row = threadIdx.x - mt * 128;
+    const uint32_t lane_base = (uint32_t)(row & ~31) << 16;
+    const uint32_t tS = tmem + lane_base + mt * 128;
+    const uint32_t tO = tmem + lane_base + 256 + mt * 128;
+    const int hh = row % g.G, tt = row / g.G;
+    long long sn = 0, on = 0;
+    bool ok = true;
+    for (long long u = blockIdx.x; u < a.num_units && ok; u += gridDim.x) {
+      Unit U;
+      if (!decode_unit(u, a, U)) continue;
+      const int qtok = (U.pair * 2 + mt) * a.Tm + tt;  // token within the query block
+      const bool valid = row < a.rows && U.i * g.B + qtok < U.len;
+      const int h = U.kvh * g.G + hh;
+      const long long orow = (long long)U.off + (long long)U.i * g.B + qtok;
+      float sl2 = a.scale_log2;
+      float vmul = 1.f;
+      if (FP8 && row < a.rows) {
+        sl2 *= __ldg(g.q_scale + h) * __ldg(g.k_scale + U.kvh);
+        vmul = __ldg(g.v_scale + U.kvh);
+      }
+      float m_ref = -INFINITY, l = 0.f;
+      for (int n = 0; n < U.count; ++n) {
+        const int j = list_entry(a, U, n);
+        ok = mbar_wait(s_full + mt, (uint32_t)(sn & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
+        if (!ok) break;
+        ++sn;
+        tc_fence_after();
+        float s[BLK];
+        {
+          uint32_t sr[BLK];
+#pragma unroll
+          for (int c = 0; c < BLK / 32; ++c) tmem_ld32(tS + c * 32, sr + c * 32);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < BLK; ++c) s[c] = __uint_as_float(sr[c]);
+        }
+        if (j == U.i) {  // diagonal block: keys after the query are masked
+#pragma unroll
+          for (int c = 0; c < BLK; ++c)
+            if (c > qtok) s[c] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int c = 1; c < BLK; ++c) mx = fmaxf(mx, s[c]);
+        const float m_new = fmaxf(m_ref, mx * sl2);
+        const bool need = m_new > m_ref + kRescaleThreshold;
+        const float f = need ? fast_exp2(m_ref - m_new) : 1.f;
+        if (need) {
+          l *= f;
+          m_ref = m_new;
+        }
+        // TMEM accesses are warp-collective: rescale when any row of the warp needs it
+        if (n > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t r16[16];
+            tmem_ld16(tO + c * 16, r16);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) r16[e] = __float_as_uint(__uint_as_float(r16[e]) * f);
+            tmem_st16(tO + c * 16, r16);
+          }
+        }
+        float lsum0 = 0.f, lsum1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < BLK; c += 2) {
+          s[c] = fast_exp2(fmaf(s[c], sl2, -m_ref));
+          s[c + 1] = fast_exp2(fmaf(s[c + 1], sl2, -m_ref));
+          lsum0 += s[c];
+          lsum1 += s[c + 1];
+        }
+        const float lsum = lsum0 + lsum1;
+        l += lsum;
+        if constexpr (!FP8) {
+#pragma unroll
+          for (int c = 0; c < BLK / 64; ++c) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(s[c * 64 + 2 * e], s[c * 64 + 2 * e + 1]);
+              pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            tmem_st32(tS + c * 32, pk);
+          }
+        } else {
+          // P = hi + lo, both e4m3: the residual plane keeps the weights' relative
+          // error near 2^-8 instead of e4m3's 2^-4.
+          uint32_t phi[BLK / 4], plo[BLK / 4];
+#pragma unroll
+          for (int e = 0; e < BLK / 4; ++e) {
+            uint32_t h32 = 0, l32 = 0;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const float x0 = s[4 * e + 2 * q], x1 = s[4 * e + 2 * q + 1];
+              const __nv_fp8x2_storage_t h = __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
+              const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(h, __NV_E4M3);
+              const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+              const __nv_fp8x2_storage_t r =
+                  __nv_cvt_float2_to_fp8x2(make_float2(x0 - hf.x, x1 - hf.y), __NV_SATFINITE, __NV_E4M3);
+              h32 |= (uint32_t)h << (16 * q);
+              l32 |= (uint32_t)r << (16 * q);
+            }
+            phi[e] = h32;
+            plo[e] = l32;
+          }
+          if constexpr (BLK / 4 == 32) {
+            tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(phi));
+            tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(plo));
+          } else {
+            tmem_st16(tS, phi);
+            tmem_st16(tS + 16, plo);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full + mt);
+      }
+      if (!ok) break;
+      // epilogue: O / l -> bf16, natural-log LSE
+      __nv_bfloat16* orow_ptr = a.o + (orow * g.Hq + h) * 128;
+      if (U.count == 0) {
+        if (valid) {
+          for (int c = 0; c < 16; ++c) reinterpret_cast<uint4*>(orow_ptr)[c] = make_uint4(0, 0, 0, 0);
+          if (a.lse) a.lse[(long long)h * a.T + orow] = -INFINITY;
+        }
+        continue;
+      }
+      ok = mbar_wait(o_full + mt, (uint32_t)(on & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
+      if (!ok) break;
+      ++on;
+      tc_fence_after();
+      const float inv = vmul / l;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r32[32];
+        tmem_ld32(tO + c * 32, r32);
+        tmem_wait_ld();
+        if (valid) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r32[2 * e]) * inv,
+                                                            __uint_as_float(r32[2 * e + 1]) * inv);
+            pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(orow_ptr + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+      }
+      if (valid && a.lse) a.lse[(long long)h * a.T + orow] = (m_ref + log2f(l)) * 0.69314718055994531f;
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool encode(CUtensorMap* m, bool fp8, int rank, const void* base, const cuuint64_t* dims, const cuuint64_t* strides,
+            const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
+            const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+template <bool FP8, int BLK, bool PAGED>
+fp_status_t run(const AttnArgs& a, const void* q, const void* k, const void* v, cudaStream_t s) {
+  using C = Cfg<FP8, BLK>;
+  const Geometry& g = a.g;
+  const cuuint64_t es = FP8 ? 1 : 2;
+  CUtensorMap mq, mk, mv;
+  {
+    const cuuint64_t dims[3] = {128, (cuuint64_t)g.Hq, (cuuint64_t)a.T};
+    const cuuint64_t strides[2] = {128 * es, (cuuint64_t)g.Hq * 128 * es};
+    const cuuint32_t box[3] = {(cuuint32_t)C::CH_ELEMS, (cuuint32_t)g.G, (cuuint32_t)a.Tm};
+    if (!encode(&mq, FP8, 3, q, dims, strides, box)) return FP_ERR_CUDA;
+  }
+  if (!PAGED) {
+    const cuuint64_t dims[3] = {128, (cuuint64_t)g.Hkv, (cuuint64_t)a.T};
+    const cuuint64_t strides[2] = {128 * es, (cuuint64_t)g.Hkv * 128 * es};
+    const cuuint32_t box[3] = {(cuuint32_t)C::CH_ELEMS, 1, (cuuint32_t)BLK};
+    if (!encode(&mk, FP8, 3, k, dims, strides, box) || !encode(&mv, FP8, 3, v, dims, strides, box))
+      return FP_ERR_CUDA;
+  } else {
+    const cuuint64_t P = (cuuint64_t)g.page_size;
+    const cuuint64_t dims[4] = {128, (cuuint64_t)g.Hkv, P, (cuuint64_t)g.num_pages};
+    const cuuint64_t strides[3] = {128 * es, (cuuint64_t)g.Hkv * 128 * es, P * g.Hkv * 128 * es};
+    const cuuint32_t box[4] = {(cuuint32_t)C::CH_ELEMS, 1, (cuuint32_t)(g.page_size < BLK ? g.page_size : BLK), 1};
+    if (!encode(&mk, FP8, 4, k, dims, strides, box) || !encode(&mv, FP8, 4, v, dims, strides, box))
+      return FP_ERR_CUDA;
+  }
+  auto kern = sparse_attention_kernel<FP8, BLK, PAGED>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+    return FP_ERR_CUDA;
+  const long long grid = a.num_units < sm_count() ? a.num_units : sm_count();
+  if (grid <= 0) return FP_OK;
+  kern<<<(unsigned)grid, kThreads, C::SMEM, s>>>(mq, mk, mv, a);
+  return cudaGetLastError() == cudaSuccess ? FP_OK : FP_ERR_CUDA;
+}
+
+}  // namespace
+
+fp_status_t launch_attention(const Geometry& g, const void* q, const void* k, const void* v, const int32_t* idx,
+                             const int32_t* cnt, void* o, float* lse, cudaStream_t s) {
+  AttnArgs a;
+  a.g = g;
+  int Tm = 1;
+  while (Tm * 2 * g.G <= 128 && Tm * 2 <= g.B) Tm *= 2;
+  const int nM = g.B / Tm;
+  if (nM < 2 || nM % 2 != 0) return FP_ERR_UNSUPPORTED;
+  a.Tm = Tm;
+  a.rows = Tm * g.G;
+  a.nPairs = nM / 2;
+  a.num_units = (long long)g.Nmax * g.R * g.Hkv * a.nPairs;
+  a.T = g.cu ? (long long)g.total_tokens : (long long)g.R * g.L;
+  a.scale_log2 = g.scale * 1.4426950408889634f;
+  a.idx = idx;
+  a.cnt = cnt;
+  a.o = reinterpret_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  const bool paged = g.page_table != nullptr;
+  if (g.B == 128) {
+    if (g.fp8) return paged ? run<true, 128, true>(a, q, k, v, s) : run<true, 128, false>(a, q, k, v, s);
+    return paged ? run<false, 128, true>(a, q, k, v, s) : run<false, 128, false>(a, q, k, v, s);
+  }
+  if (g.B == 64) {
+    if (g.fp8) return paged ? run<true, 64, true>(a, q, k, v, s) : run<true, 64, false>(a, q, k, v, s);
+    return paged ? run<false, 64, true>(a, q, k, v, s) : run<false, 64, false>(a, q, k, v, s);
+  }
+  return FP_ERR_UNSUPPORTED;
+}
+
+}  // namespace fp

@@ -1,0 +1,75 @@
+// Internal (non-ABI) definitions shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "flashprefill.h"
+
+namespace fp {
+
+// Validated, derived geometry of one call. Built on the host from fp_params_t.
+struct Geometry {
+  int R;          // requests (batch)
+  int L;          // max_seqlen (contiguous: every request's length)
+  int Hq, Hkv, G, d;
+  int B;          // block size (tokens)
+  int Nmax;       // ceil(L / B)
+  int Wmax;       // ceil(Nmax / 32) mask words per row
+  int Npad;       // Nmax rounded up to a multiple of 4 (stride of the transposed pooled K)
+  int Sb, Wb;     // sink / window in blocks
+  float scale;    // softmax scale
+  float thr;      // ln(alpha) (-inf for alpha == 0)
+  int fp8;        // Q/K/V are e4m3
+  const int32_t* cu;        // device cu_seqlens or nullptr
+  int total_tokens;
+  const int32_t* page_table;  // device or nullptr
+  int page_size, page_shift, max_pages, num_pages;
+  const float* q_scale;
+  const float* k_scale;
+  const float* v_scale;
+  unsigned* status;         // device status word
+};
+
+// Start token (row of the packed/contiguous layout) and length of request r.
+// Invalid cu_seqlens make the request empty and set FP_DEV_BAD_SEQLENS.
+__device__ __forceinline__ void request_span(const Geometry& g, int r, int& off, int& len) {
+  if (g.cu == nullptr) {
+    off = r * g.L;
+    len = g.L;
+    return;
+  }
+  const int a = __ldg(g.cu + r), b = __ldg(g.cu + r + 1);
+  if (a < 0 || b < a || b - a > g.L || b > g.total_tokens) {
+    atomicOr(g.status, FP_DEV_BAD_SEQLENS);
+    off = 0;
+    len = 0;
+    return;
+  }
+  off = a;
+  len = b - a;
+}
+
+__host__ __device__ __forceinline__ long long list_row_base(int r, int kvh, int i, int Hkv, int Nmax) {
+  return ((long long)r * Hkv + kvh) * ((long long)Nmax * (Nmax + 1) / 2) + (long long)i * (i + 1) / 2;
+}
+
+__host__ __device__ __forceinline__ long long row_index(int r, int kvh, int i, int Hkv, int Nmax) {
+  return ((long long)r * Hkv + kvh) * Nmax + i;
+}
+
+// host launchers (each returns a cudaError_t of its launch)
+cudaError_t launch_pool(const Geometry& g, const void* q, const void* k, float* qbar, float* kbarT,
+                        cudaStream_t s);
+cudaError_t launch_score(const Geometry& g, const float* qbar, const float* kbarT, uint32_t* mask,
+                         int32_t* idx, int32_t* cnt, cudaStream_t s);
+cudaError_t launch_compact(const Geometry& g, const uint32_t* mask, int32_t* idx, int32_t* cnt,
+                           cudaStream_t s);
+// Returns FP_OK, FP_ERR_UNSUPPORTED or FP_ERR_CUDA.
+fp_status_t launch_attention(const Geometry& g, const void* q, const void* k, const void* v,
+                             const int32_t* idx, const int32_t* cnt, void* o, float* lse,
+                             cudaStream_t s);
+
+size_t score_smem_bytes(const Geometry& g);
+
+}  // namespace fp

@@ -1,0 +1,177 @@
+/*
+ * flashprefill.h -- C ABI of the B200 (sm_100a) block-sparse causal prefill
+ * attention library (FlashPrefill style).
+ *
+ * The method (sources: "FlashPrefill: Near-Zero-Cost Sparsity Discovery for
+ * Ultra-Fast Long-Context Prefilling", zhichai.net summary, Method 1-3, and the
+ * "FlashPrefill V2: Block-Sparse Prefill Attention for Long-Context LLM Serving"
+ * abstract):
+ *   1. fp_discover  -- mean-pool Q and K per block of B tokens, score every
+ *      causal pair of pooled blocks, keep a block when exp(score - row max) >=
+ *      alpha (per query head, union over the KV group's heads), always keep the
+ *      sink and local-window blocks; emit a bit mask.
+ *   2. fp_compact   -- turn each mask row into a contiguous ascending list of
+ *      kept block indices ("index compaction -> physical jumps").
+ *   3. fp_sparse_prefill / fp_paged_sparse_prefill -- flash attention with
+ *      online softmax that visits only the listed KV blocks; all query heads of
+ *      a KV group share each K/V tile (PackGQA); BF16 or FP8-e4m3; contiguous,
+ *      varlen (continuous batching) or paged KV.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *   allocates nothing and keeps no per-call state. Pointers to Q/K/V/O and to
+ *   pools must be 16-byte aligned.
+ * - Every call is asynchronous on the given CUDA stream (cudaStream_t, passed
+ *   as void*; NULL = legacy default stream). Argument errors are returned
+ *   before anything is launched. FP_ERR_CUDA reports a launch error.
+ *   Device-side checks (bad cu_seqlens, page id or list entry, a pipeline wait
+ *   that exceeded its time limit) never trap: they set a device status word
+ *   that fp_get_device_status() reads and clears.
+ * - Sequences ("requests") r = 0..R-1. Without cu_seqlens the batch is
+ *   contiguous: R = batch, every request has max_seqlen tokens, Q is
+ *   [R, L, Hq, d] and K/V are [R, L, Hkv, d] (row-major, d innermost). With
+ *   cu_seqlens (device int32 [R+1], non-decreasing, cu[0] = 0,
+ *   cu[R] = total_tokens) request r owns tokens cu[r] .. cu[r+1]-1 of a packed
+ *   Q [total_tokens, Hq, d] (and of K/V [total_tokens, Hkv, d] when not
+ *   paged); every length must be <= max_seqlen.
+ * - Paged KV (page_table != NULL, requires cu_seqlens): K/V live in pools
+ *   [num_pages, page_size, Hkv, d]; token t of request r is slot t % page_size
+ *   of pool page page_table[r * max_pages_per_req + t / page_size].
+ * - Block grid: per request, blocks of B = block tokens start at the request's
+ *   first token; N_r = ceil(L_r / B); Nmax = ceil(max_seqlen / B). Query head h
+ *   uses KV head h / G with G = Hq / Hkv.
+ * - Mask layout (uint32): word w of row (r, g, i) is
+ *   mask[((r * Hkv + g) * Nmax + i) * Wmax + w], Wmax = ceil(Nmax / 32); bit b
+ *   of word w is key block j = 32 w + b. Only j <= i can be set.
+ * - List layout (int32): row (r, g, i) starts at
+ *   idx[(r * Hkv + g) * Nmax * (Nmax + 1) / 2 + i * (i + 1) / 2] and holds
+ *   cnt[(r * Hkv + g) * Nmax + i] strictly ascending block indices (capacity
+ *   i + 1). Rows i >= N_r have cnt = 0.
+ * - Thresholding happens in float32: keep iff s - rowmax >= ln(alpha), with
+ *   s = softmax_scale * (pooled q . pooled k). Blocks whose exact probability
+ *   lies within ~1e-5 relative of alpha may be decided either way.
+ */
+#ifndef FLASHPREFILL_H_
+#define FLASHPREFILL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FP_OK = 0,
+  FP_ERR_INVALID_ARG = -1,  /* null pointer, bad size, alpha < 0 or not finite */
+  FP_ERR_UNSUPPORTED = -2,  /* head_dim != 128, block not 64/128, unsupported G */
+  FP_ERR_ALIGNMENT = -3,    /* a tensor pointer is not 16-byte aligned */
+  FP_ERR_WORKSPACE = -4,    /* workspace missing or smaller than fp_workspace_size */
+  FP_ERR_CUDA = -5,         /* a CUDA runtime call or launch failed */
+  FP_ERR_DEVICE = -6        /* the device status word is non-zero (see fp_get_device_status) */
+} fp_status_t;
+
+typedef enum { FP_BF16 = 0, FP_E4M3 = 1 } fp_dtype_t;
+
+/* Device status bits (fp_get_device_status). */
+#define FP_DEV_TIMEOUT 0x1u       /* a pipeline wait exceeded its limit; outputs invalid */
+#define FP_DEV_BAD_SEQLENS 0x2u   /* cu_seqlens not monotone / out of range */
+#define FP_DEV_BAD_PAGE 0x4u      /* page id outside [0, num_pages) */
+#define FP_DEV_BAD_LIST 0x8u      /* list entry outside [0, i] or count > i+1 */
+
+typedef struct {
+  fp_dtype_t dtype;        /* element type of Q, K, V (O is always bf16) */
+  int batch;               /* contiguous layout: number of sequences; varlen: number of requests R */
+  int max_seqlen;          /* contiguous: tokens per sequence; varlen: upper bound on every length */
+  int hq, hkv;             /* query heads, KV heads; hq % hkv == 0 */
+  int head_dim;            /* must be 128 */
+  int block;               /* B: 64 or 128 tokens */
+  float alpha;             /* dynamic-threshold factor, finite and >= 0 */
+  int sink_tokens;         /* leading tokens always kept: ceil(sink_tokens / B) blocks */
+  int window_tokens;       /* local window: max(1, ceil(window_tokens / B)) blocks ending at the diagonal */
+  float softmax_scale;     /* 0 -> 1 / sqrt(head_dim); used for scores and attention */
+  const float* q_scale;    /* FP8 only: device float [hq], dequantisation scale per query head */
+  const float* k_scale;    /* FP8 only: device float [hkv] */
+  const float* v_scale;    /* FP8 only: device float [hkv] */
+  const int32_t* cu_seqlens;  /* device int32 [batch + 1] or NULL (contiguous batch) */
+  int total_tokens;           /* varlen: cu_seqlens[batch] (rows of the packed Q) */
+  const int32_t* page_table;  /* device int32 [batch, max_pages_per_req] or NULL */
+  int page_size;              /* paged: tokens per page (power of two, 16..256) */
+  int max_pages_per_req;
+  int num_pages;              /* paged: pages in each pool */
+} fp_params_t;
+
+/* Bytes of device scratch fp_discover needs (pooled Q and K, float32). */
+size_t fp_workspace_size(const fp_params_t* p);
+/* Number of uint32 words of the block mask: R * Hkv * Nmax * ceil(Nmax / 32). */
+size_t fp_mask_words(const fp_params_t* p);
+/* Number of int32 entries of the index lists: R * Hkv * Nmax * (Nmax + 1) / 2. */
+size_t fp_list_capacity(const fp_params_t* p);
+/* Number of int32 row counts: R * Hkv * Nmax. */
+size_t fp_count_entries(const fp_params_t* p);
+
+/*
+ * Block pattern discovery (Method 1 "Instantaneous Pattern Discovery" and
+ * Method 2 "Dynamic Threshold Pruning" of the FlashPrefill summary).
+ * q: Q (bf16 or e4m3 per p->dtype, layout above); k: K, or the K pool when
+ * p->page_table is set. mask: device uint32 [fp_mask_words(p)], fully
+ * written (rows i >= N_r are zero). workspace: device scratch of
+ * ws_bytes >= fp_workspace_size(p), 256-byte aligned; contents are
+ * overwritten.
+ */
+fp_status_t fp_discover(const fp_params_t* p, const void* q, const void* k, uint32_t* mask,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Index compaction (Method 3 "Index Compaction -> Physical Jumps"): mask ->
+ * ascending lists. idx: device int32 [fp_list_capacity(p)]; cnt: device int32
+ * [fp_count_entries(p)], fully written.
+ */
+fp_status_t fp_compact(const fp_params_t* p, const uint32_t* mask, int32_t* idx, int32_t* cnt,
+                       void* stream);
+
+/*
+ * Discovery and compaction in one pass over the pooled scores: same outputs as
+ * fp_discover followed by fp_compact (mask may be NULL to skip writing it).
+ */
+fp_status_t fp_discover_compact(const fp_params_t* p, const void* q, const void* k,
+                                uint32_t* mask, int32_t* idx, int32_t* cnt, void* workspace,
+                                size_t ws_bytes, void* stream);
+
+/*
+ * Block-sparse flash attention over the compacted lists ("FlashPrefill V2"
+ * abstract: PackGQA, warp specialisation, ping-pong pipelining, FP8).
+ * For each request r, query token t and head h:
+ *   O[t, h] = sum_k softmax_k(scale * q_t,h . k_k) v_k over the keys k <= t of
+ *   the blocks listed in row (r, h / G, t / B).
+ * q, k, v: contiguous or varlen layout (no page table; p->page_table must be
+ * NULL). o: device bf16, same layout as q. lse: NULL or device float
+ * [hq, R * max_seqlen] (contiguous) / [hq, total_tokens] (varlen), natural-log
+ * sum of exponentials of the scaled logits. Rows with cnt = 0 get O = 0 and
+ * lse = -inf. Output rows of tokens outside every request are not written.
+ */
+fp_status_t fp_sparse_prefill(const fp_params_t* p, const void* q, const void* k, const void* v,
+                              const int32_t* idx, const int32_t* cnt, void* o, float* lse,
+                              void* stream);
+
+/* As fp_sparse_prefill, with K/V read through p->page_table from the pools. */
+fp_status_t fp_paged_sparse_prefill(const fp_params_t* p, const void* q, const void* k_pool,
+                                    const void* v_pool, const int32_t* idx, const int32_t* cnt,
+                                    void* o, float* lse, void* stream);
+
+/*
+ * Synchronises `stream`, writes the device status bits (FP_DEV_*) of the
+ * current device to *bits (may be NULL) and clears them. Returns FP_OK if no
+ * bit was set, FP_ERR_DEVICE otherwise, FP_ERR_CUDA on a runtime error.
+ */
+fp_status_t fp_get_device_status(uint32_t* bits, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* fp_status_string(fp_status_t s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLASHPREFILL_H_ */

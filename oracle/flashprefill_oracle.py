@@ -65,7 +65,7 @@ import numpy as np
 
 __all__ = [
     "num_blocks", "forced_blocks", "pool_blocks", "pooled_scores", "head_keep",
-    "block_mask", "compact", "attention_rows", "block_sparse_attention",
+    "block_mask", "discover_row", "compact", "attention_rows", "block_sparse_attention",
     "flashprefill", "gather_pages", "flashprefill_paged", "row_borderline",
 ]
 
@@ -133,6 +133,22 @@ def block_mask(qbar, kbar, scale: float, alpha: float, Sb: int, Wb: int) -> np.n
     forced = (j <= i) & ((j < Sb) | (i - j < Wb))
     mask |= forced[None]
     return mask
+
+
+def discover_row(qbar_i: np.ndarray, kbar_g: np.ndarray, i: int, scale: float, alpha: float,
+                 Sb: int, Wb: int) -> np.ndarray:
+    """Kept blocks of one (KV group, query block i) row, computed on its own:
+    qbar_i [G, d] are the pooled queries of the group's heads at block i,
+    kbar_g [N, d] the group's pooled keys. Same steps as ``block_mask`` (per-head
+    threshold against the head's row max, union, sink/window), then the
+    ascending list of kept j."""
+    s = scale * (qbar_i @ kbar_g[: i + 1].T)  # [G, i+1]
+    keep = np.zeros(i + 1, dtype=bool)
+    for h in range(s.shape[0]):
+        keep |= np.exp(s[h] - s[h].max()) >= alpha
+    j = np.arange(i + 1)
+    keep |= (j < Sb) | (i - j < Wb)
+    return np.flatnonzero(keep)
 
 
 def compact(mask: np.ndarray):

@@ -1,0 +1,279 @@
+"""GPU parity of the CUDA path (through the C ABI) against the float64 oracle.
+
+Discovery + compaction: kept-block lists bit-exact except borderline blocks
+(exact probability within 1e-5 relative of alpha). Attention: run on the
+oracle's own lists; BF16 max |err| <= 2e-2, mean <= 2e-3; FP8 max <= 6e-2.
+Small cases span several tiles and a ragged tail; the full-size workloads are
+checked on sampled query blocks.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_long_blocks_b200 import workloads as wl
+from tests import _helpers as H
+
+pytestmark = pytest.mark.gpu
+
+W = wl.workloads()
+
+
+def _case(name, L=None, **kw):
+    w = W[name]
+    if L is not None:
+        w = wl.small_case(w, L)
+    return w.with_(**kw) if kw else w
+
+
+def _inputs(w, fp8=False):
+    inp = wl.make_inputs(w)
+    return wl.to_fp8(inp) if fp8 else inp
+
+
+def _mask_matches_lists(dev):
+    m = dev.mask()
+    lists = dev.lists()
+    for r in range(dev.cfg.batch):
+        for g in range(dev.cfg.hkv):
+            for i in range(dev.cfg.nmax):
+                assert np.flatnonzero(m[r, g, i]).tolist() == lists[r][g][i]
+
+
+# ----------------------------------------------------------------------------- discovery
+DISCOVERY_CASES = [
+    ("tiny2k", None, None),
+    ("qwen7b_32k", 4096, 0.0),
+    ("qwen7b_32k", 4096, 0.05),
+    ("qwen7b_32k", 5000, 0.2),
+    ("qwen30b_128k", 8192, None),
+    ("qwen30b_128k", 3000, 1.0),
+    ("extreme_256k", 8192, None),
+    ("extreme_256k", 1000, 3.0),
+]
+
+
+@pytest.mark.parametrize("name,L,alpha", DISCOVERY_CASES)
+@pytest.mark.parametrize("fused", [True, False])
+def test_discovery_matches_oracle(name, L, alpha, fused):
+    w = _case(name, L)
+    inp = _inputs(w)
+    dev = H.Device(w, inp, alpha)
+    dev.discover(fused=fused)
+    assert dev.status() == 0
+    orc = H.oracle_discovery(w, inp, alpha)
+    H.compare_lists(orc, dev.lists())
+    _mask_matches_lists(dev)
+
+
+@pytest.mark.parametrize("name,L", [("tiny2k", None), ("qwen30b_128k", 4096)])
+def test_discovery_fp8_matches_oracle(name, L):
+    w = _case(name, L)
+    inp = _inputs(w, fp8=True)
+    dev = H.Device(w, inp)
+    dev.discover()
+    assert dev.status() == 0
+    H.compare_lists(H.oracle_discovery(w, inp), dev.lists())
+
+
+def test_discovery_alpha_zero_and_above_one():
+    w = _case("qwen30b_128k", 2000)
+    inp = _inputs(w)
+    for alpha, expect in [(0.0, "all"), (1.5, "forced")]:
+        dev = H.Device(w, inp, alpha)
+        dev.discover()
+        lists = dev.lists()[0]
+        N = dev.cfg.nmax
+        Sb, Wb = oracle.forced_blocks(w.sink_tokens, w.window_tokens, w.block)
+        for g in range(w.hkv):
+            for i in range(N):
+                want = list(range(i + 1)) if expect == "all" else \
+                    [j for j in range(i + 1) if j < Sb or i - j < Wb]
+                assert lists[g][i] == want
+
+
+# ----------------------------------------------------------------------------- attention
+ATTN_CASES = [
+    ("tiny2k", None, None),              # B=64, G=4, full size
+    ("qwen7b_32k", 2048, 0.0),           # G=7 (112-row M-tiles), alpha=0: dense causal
+    ("qwen30b_128k", 3000, None),        # G=8, ragged tail
+    ("qwen30b_128k", 4096, 0.3),
+    ("extreme_256k", 2500, None),
+    ("qwen30b_128k", 100, None),         # one partial block
+]
+
+
+@pytest.mark.parametrize("name,L,alpha", ATTN_CASES)
+@pytest.mark.parametrize("fp8", [False, True])
+def test_attention_on_oracle_lists(name, L, alpha, fp8):
+    w = _case(name, L)
+    inp = _inputs(w, fp8)
+    dev = H.Device(w, inp, alpha)
+    orc = H.oracle_discovery(w, inp, alpha)
+    idx, cnt = H.upload_lists(dev.cfg, [o["lists"] for o in orc])
+    dev.attend(idx, cnt)
+    assert dev.status() == 0
+    H.check_attention(dev, H.oracle_attention(w, inp, orc), fp8)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_full_path_tiny(fp8):
+    """Discovery -> compaction -> attention on the GPU; lists equal the oracle's."""
+    w = _case("tiny2k")
+    inp = _inputs(w, fp8)
+    dev = H.Device(w, inp)
+    dev.discover()
+    orc = H.oracle_discovery(w, inp)
+    assert H.compare_lists(orc, dev.lists()) == 0
+    dev.attend()
+    assert dev.status() == 0
+    H.check_attention(dev, H.oracle_attention(w, inp, orc), fp8)
+
+
+def test_values_ones_and_zero_queries():
+    """V = 1 gives O = 1; Q = 0 gives the mean of V over the allowed keys (alpha = 0)."""
+    w = _case("qwen30b_128k", 1000)
+    inp = _inputs(w)
+    inp.v = torch.ones_like(inp.v)
+    dev = H.Device(w, inp, 0.0)
+    dev.discover()
+    dev.attend()
+    o = dev.bufs.o.float()
+    assert (o - 1).abs().max().item() <= 1e-2
+    inp2 = _inputs(w)
+    inp2.q = torch.zeros_like(inp2.q)
+    dev2 = H.Device(w, inp2, 0.0)
+    dev2.discover()
+    dev2.attend()
+    v = inp2.v[0, :, 0].double()
+    ref = torch.cumsum(v, 0) / torch.arange(1, v.shape[0] + 1, dtype=torch.float64)[:, None]
+    got = dev2.bufs.o[0, :, 0].double().cpu()
+    assert (got - ref).abs().max().item() <= 2e-2
+
+
+def test_empty_rows_give_zero_output():
+    w = _case("qwen30b_128k", 512)
+    inp = _inputs(w)
+    dev = H.Device(w, inp)
+    N = dev.cfg.nmax
+    lists = [[[list(range(i + 1)) if i != 2 else [] for i in range(N)] for _ in range(w.hkv)]]
+    idx, cnt = H.upload_lists(dev.cfg, lists)
+    dev.attend(idx, cnt)
+    o = dev.bufs.o[0].float()
+    assert o[256:384].abs().max().item() == 0.0
+    assert torch.isinf(dev.bufs.lse[:, 256:384]).all()
+    assert torch.isfinite(o).all()
+
+
+# ----------------------------------------------------------------------------- paged / varlen
+@pytest.mark.parametrize("fp8", [False, True])
+def test_paged_varlen_matches_oracle(fp8):
+    w = W["paged_varlen"].with_(seqlens=(700, 1290, 64, 2048))
+    inp = _inputs(w, fp8)
+    dev = H.Device(w, inp)
+    dev.discover()
+    assert dev.status() == 0
+    orc = H.oracle_discovery(w, inp)
+    H.compare_lists(orc, dev.lists())
+    dev.attend()
+    assert dev.status() == 0
+    H.check_attention(dev, H.oracle_attention(w, inp, orc), fp8)
+
+
+def test_paged_identity_table_equals_permuted():
+    """Permuting the pool and the table together leaves every output bit unchanged."""
+    w = W["paged_varlen"].with_(seqlens=(1000, 333, 1500))
+    inp = _inputs(w)
+    dev = H.Device(w, inp)
+    dev.discover()
+    dev.attend()
+    o1, l1 = dev.bufs.o.clone(), dev.bufs.lse.clone()
+    n = inp.k_pool.shape[0]
+    perm = torch.randperm(n, generator=torch.Generator().manual_seed(9))
+    inv = torch.empty_like(perm)
+    inv[perm] = torch.arange(n)
+    inp2 = wl.Inputs(w, inp.q, cu_seqlens=inp.cu_seqlens, k_pool=inp.k_pool[inv], v_pool=inp.v_pool[inv],
+                     page_table=torch.where(inp.page_table >= 0, perm[inp.page_table.long().clamp(min=0)].int(),
+                                            inp.page_table))
+    dev2 = H.Device(w, inp2)
+    dev2.discover()
+    dev2.attend()
+    assert torch.equal(o1, dev2.bufs.o) and torch.equal(l1, dev2.bufs.lse)
+    assert torch.equal(dev.bufs.cnt, dev2.bufs.cnt)
+
+
+def test_single_request_paged_equals_contiguous():
+    L = 1500
+    wc = _case("qwen30b_128k", L)
+    inc = _inputs(wc)
+    dc = H.Device(wc, inc)
+    dc.discover()
+    dc.attend()
+    wp = W["paged_varlen"].with_(seqlens=(L,), hkv=4, seed=wc.seed, seed_stride=0, heavy_frac=wc.heavy_frac,
+                                  n_slash=wc.n_slash, amp_scale=wc.amp_scale)
+    inpp = _inputs(wp)
+    assert torch.equal(inpp.q, inc.q[0])
+    dp = H.Device(wp, inpp)
+    dp.discover()
+    dp.attend()
+    assert torch.equal(dc.bufs.cnt, dp.bufs.cnt)
+    assert torch.equal(dc.bufs.o[0], dp.bufs.o)
+
+
+# ----------------------------------------------------------------------------- device checks
+def test_bad_page_and_list_entries_are_reported():
+    w = W["paged_varlen"].with_(seqlens=(600, 300))
+    inp = _inputs(w)
+    inp.page_table = inp.page_table.clone()
+    inp.page_table[0, 3] = 10_000  # outside the pool
+    dev = H.Device(w, inp)
+    dev.discover()
+    assert dev.status() & 4  # FP_DEV_BAD_PAGE
+    dev.attend()
+    assert dev.status() & 4
+    w2 = _case("qwen30b_128k", 512)
+    dev2 = H.Device(w2, _inputs(w2))
+    N = dev2.cfg.nmax
+    lists = [[[[i + 1] if i == 1 else list(range(i + 1)) for i in range(N)] for _ in range(w2.hkv)]]
+    idx, cnt = H.upload_lists(dev2.cfg, lists)
+    dev2.attend(idx, cnt)
+    assert dev2.status() & 8  # FP_DEV_BAD_LIST
+    assert dev2.status() == 0  # cleared by the read
+
+
+def test_bad_cu_seqlens_reported():
+    w = W["paged_varlen"].with_(seqlens=(600, 300))
+    inp = _inputs(w)
+    inp.cu_seqlens = torch.tensor([0, 600, 500], dtype=torch.int32)  # decreasing
+    dev = H.Device(w, inp)
+    dev.discover()
+    assert dev.status() & 2  # FP_DEV_BAD_SEQLENS
+
+
+# ----------------------------------------------------------------------------- full sizes (sampled)
+def _sample_rows(orc, w, r=0, k=6, seed=0):
+    N = orc[r]["mask"].shape[1]
+    dens = orc[r]["cnt"].sum(axis=0)
+    rng = np.random.default_rng(seed)
+    picks = {0, N - 1, N // 2, int(np.argmax(dens))} | set(rng.integers(0, N, k).tolist())
+    g_pick = rng.integers(0, w.hkv, len(picks)).tolist()
+    return {(r, g, i) for g, i in zip(g_pick, sorted(picks))}
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_full_size_128k(fp8):
+    w = W["qwen30b_128k"]
+    inp = _inputs(w, fp8)
+    dev = H.Device(w, inp)
+    dev.discover()
+    assert dev.status() == 0
+    orc = H.oracle_discovery(w, inp)
+    rep = {}
+    H.compare_lists(orc, dev.lists(), rep)
+    print("128K borderline blocks:", rep)
+    idx, cnt = H.upload_lists(dev.cfg, [o["lists"] for o in orc])
+    dev.attend(idx, cnt)
+    assert dev.status() == 0
+    rows = _sample_rows(orc, w)
+    H.check_attention(dev, H.oracle_attention(w, inp, orc, rows), fp8, rep)
+    print("128K attention:", rep)

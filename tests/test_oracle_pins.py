@@ -401,3 +401,15 @@ def test_planted_mistake_fails_a_pin(monkeypatch, name, func):
     monkeypatch.setattr(fo, name, func)
     monkeypatch.setattr(oracle, name, func, raising=False)
     assert not _pins_pass(), f"mutation of {name} ({func.__name__}) went unnoticed"
+
+
+def test_discover_row_agrees_with_block_mask():
+    """The per-row entry point (used to time bounded samples) takes the same steps."""
+    Q, K, V = _rand(96, 8, 2, 8, 31, amp=3.0)
+    B, a, sink, win = 8, 0.2, 8, 16
+    r = oracle.flashprefill(Q, K, V, B, a, sink, win, attention=False)
+    Sb, Wb = oracle.forced_blocks(sink, win, B)
+    for g in range(2):
+        for i in range(12):
+            got = oracle.discover_row(r["qbar"][i, 4 * g: 4 * g + 4], r["kbar"][:, g], i, r["scale"], a, Sb, Wb)
+            np.testing.assert_array_equal(got, np.flatnonzero(r["mask"][g, i]))
