@@ -26,7 +26,10 @@ DEV_TIMEOUT, DEV_BAD_SEQLENS, DEV_BAD_PAGE, DEV_BAD_LIST = 1, 2, 4, 8
 
 class FPError(RuntimeError):
     def __init__(self, fn: str, code: int):
-        super().__init__(f"{fn} returned {STATUS.get(code, code)}")
+        detail = ""
+        if code == -5 and _lib is not None:
+            detail = " (" + (_lib.fp_last_error() or b"").decode(errors="replace") + ")"
+        super().__init__(f"{fn} returned {STATUS.get(code, code)}{detail}")
         self.code = code
 
 
@@ -82,6 +85,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "fp_paged_sparse_prefill": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
         "fp_get_device_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), vp]),
         "fp_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "fp_last_error": (ctypes.c_char_p, []),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)

@@ -1,6 +1,7 @@
 // C ABI entry points: argument validation, derived geometry, workspace layout,
 // launches on the caller's stream, and the device status word.
 #include <cmath>
+#include <cstdio>
 #include <cstdint>
 #include <mutex>
 
@@ -11,9 +12,20 @@ namespace fp {
 // Device-side error bits (FP_DEV_*); set by kernels, read/cleared by fp_get_device_status.
 __device__ unsigned g_device_status;
 
+thread_local char t_last_error[256] = "";
+
+void set_last_error(const char* step, int code, const char* detail) {
+  snprintf(t_last_error, sizeof(t_last_error), "%s failed (code %d): %s", step, code, detail ? detail : "");
+}
+
 namespace {
 
 constexpr int kMaxDevices = 64;
+
+fp_status_t cuda_fail(const char* step, cudaError_t e) {
+  set_last_error(step, (int)e, cudaGetErrorString(e));
+  return FP_ERR_CUDA;
+}
 
 unsigned* status_ptr() {
   static unsigned* ptrs[kMaxDevices] = {};
@@ -117,12 +129,14 @@ fp_status_t discover_impl(const fp_params_t* p, const void* q, const void* k, ui
   Geometry g = geometry(p);
   if (score_smem_bytes(g) > 227 * 1024) return FP_ERR_UNSUPPORTED;
   g.status = status_ptr();
-  if (!g.status) return FP_ERR_CUDA;
+  if (!g.status) return cuda_fail("device status symbol", cudaGetLastError());
   float* qbar = static_cast<float*>(ws);
   float* kbarT = qbar + (qbar_floats(g) + 63) / 64 * 64;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (launch_pool(g, q, k, qbar, kbarT, s) != cudaSuccess) return FP_ERR_CUDA;
-  if (launch_score(g, qbar, kbarT, mask, idx, cnt, s) != cudaSuccess) return FP_ERR_CUDA;
+  cudaError_t e = launch_pool(g, q, k, qbar, kbarT, s);
+  if (e != cudaSuccess) return cuda_fail("pool launch", e);
+  e = launch_score(g, qbar, kbarT, mask, idx, cnt, s);
+  if (e != cudaSuccess) return cuda_fail("score launch", e);
   return FP_OK;
 }
 
@@ -137,7 +151,7 @@ fp_status_t attention_impl(const fp_params_t* p, bool paged, const void* q, cons
     return FP_ERR_ALIGNMENT;
   Geometry g = geometry(p);
   g.status = status_ptr();
-  if (!g.status) return FP_ERR_CUDA;
+  if (!g.status) return cuda_fail("device status symbol", cudaGetLastError());
   return launch_attention(g, q, k, v, idx, cnt, o, lse, static_cast<cudaStream_t>(stream));
 }
 
@@ -191,9 +205,9 @@ fp_status_t fp_compact(const fp_params_t* p, const uint32_t* mask, int32_t* idx,
   if (!aligned(mask, 4) || !aligned(idx, 4) || !aligned(cnt, 4)) return FP_ERR_ALIGNMENT;
   Geometry g = geometry(p);
   g.status = status_ptr();
-  if (!g.status) return FP_ERR_CUDA;
-  return launch_compact(g, mask, idx, cnt, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FP_OK
-                                                                                              : FP_ERR_CUDA;
+  if (!g.status) return cuda_fail("device status symbol", cudaGetLastError());
+  const cudaError_t e = launch_compact(g, mask, idx, cnt, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FP_OK : cuda_fail("compact launch", e);
 }
 
 fp_status_t fp_sparse_prefill(const fp_params_t* p, const void* q, const void* k, const void* v, const int32_t* idx,
@@ -209,13 +223,17 @@ fp_status_t fp_paged_sparse_prefill(const fp_params_t* p, const void* q, const v
 fp_status_t fp_get_device_status(uint32_t* bits, void* stream) {
   unsigned* sp = status_ptr();
   if (!sp) return FP_ERR_CUDA;
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP_ERR_CUDA;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail("stream synchronize", e);
   unsigned v = 0;
-  if (cudaMemcpy(&v, sp, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return FP_ERR_CUDA;
-  if (v && cudaMemset(sp, 0, sizeof(unsigned)) != cudaSuccess) return FP_ERR_CUDA;
+  e = cudaMemcpy(&v, sp, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail("status read", e);
+  if (v && (e = cudaMemset(sp, 0, sizeof(unsigned))) != cudaSuccess) return cuda_fail("status clear", e);
   if (bits) *bits = v;
   return v ? FP_ERR_DEVICE : FP_OK;
 }
+
+const char* fp_last_error(void) { return t_last_error; }
 
 const char* fp_status_string(fp_status_t s) {
   switch (s) {

@@ -11,12 +11,13 @@
 // that Tm * G <= 128, so every K/V tile a CTA loads serves all G heads. A CTA
 // owns two M-tiles (ping-pong) and walks row (r, kvh, i)'s list.
 //
-// Roles (320 threads, one persistent CTA per SM):
+// Roles (384 threads, one persistent CTA per SM):
 //   warps 0-3  softmax warpgroup for M-tile 0 (one thread per row)
 //   warps 4-7  softmax warpgroup for M-tile 1
 //   warp 8     TMA producer: Q tiles, then K[idx[n]] and V[idx[n]] into rings
 //   warp 9     MMA issuer (one thread): S = Q K^T into TMEM, O += P V with P
 //              read from TMEM (aliasing S), accumulators in TMEM
+//   warps 10-11 idle (complete the third warpgroup for the register split)
 // Order of MMAs per visit n (ping-pong): PV0(n), S0(n+1), PV1(n), S1(n+1), so
 // one warpgroup's softmax overlaps the other tile's MMAs.
 // Softmax: online, base-2, with the running reference max raised only when the
@@ -27,6 +28,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include <cstdio>
 #include <mutex>
 
 #include "internal.cuh"
@@ -36,9 +38,16 @@ namespace fp {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;  // 3 warpgroups
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+// Launched at 168 registers/thread (384 x 168 = 64512). The softmax warpgroups
+// then raise their limit and the producer/MMA warpgroup lowers its own:
+// 2 x 128 x 200 + 128 x 96 = 63488 <= 64512, and per SM sub-partition (three
+// warps each) 2 x 32 x 200 + 32 x 96 = 15872 <= 16384.
+constexpr uint32_t kSoftmaxRegs = 200;
+constexpr uint32_t kControlRegs = 96;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * 168, "register split exceeds the launch");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kSmemBudget = 200 * 1024;
 
@@ -152,7 +161,7 @@ __device__ __forceinline__ void load_kv_tile(uint8_t* dst, const CUtensorMap* ma
 }
 
 template <bool FP8, int BLK, bool PAGED>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kThreads, 1)
     sparse_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   using C = Cfg<FP8, BLK>;
@@ -215,6 +224,7 @@ __global__ void __maxnreg__(200)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp >= 8) reg_dealloc<kControlRegs>();
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
@@ -362,8 +372,9 @@ __global__ void __maxnreg__(200)
       int never = 0;
       mbar_wait(drain, 0u, (volatile int*)&never, g.status, FP_DEV_TIMEOUT);
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax warpgroups
+    reg_alloc<kSoftmaxRegs>();
     const int mt = warp >> 2;
     const int row = threadIdx.x - mt * 128;
     const uint32_t lane_base = (uint32_t)(row & ~31) << 16;
@@ -549,12 +560,23 @@ EncodeTiledFn encode_fn() {
 bool encode(CUtensorMap* m, bool fp8, int rank, const void* base, const cuuint64_t* dims, const cuuint64_t* strides,
             const cuuint32_t* box) {
   EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
+  if (!fn) {
+    set_last_error("cuTensorMapEncodeTiled lookup", 0, "driver entry point not found");
+    return false;
+  }
   cuuint32_t es[4] = {1, 1, 1, 1};
-  return fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
-            const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const CUresult r = fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
+                        const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[160];
+    snprintf(buf, sizeof(buf), "rank %d dims %llu,%llu,%llu box %u,%u,%u", rank, (unsigned long long)dims[0],
+             (unsigned long long)dims[1], (unsigned long long)dims[2], box[0], box[1], box[2]);
+    set_last_error("cuTensorMapEncodeTiled", (int)r, buf);
+    return false;
+  }
+  return true;
 }
 
 int sm_count() {
@@ -591,12 +613,20 @@ fp_status_t run(const AttnArgs& a, const void* q, const void* k, const void* v, 
       return FP_ERR_CUDA;
   }
   auto kern = sparse_attention_kernel<FP8, BLK, PAGED>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) {
+    set_last_error("attention smem attribute", (int)e, cudaGetErrorString(e));
     return FP_ERR_CUDA;
+  }
   const long long grid = a.num_units < sm_count() ? a.num_units : sm_count();
   if (grid <= 0) return FP_OK;
   kern<<<(unsigned)grid, kThreads, C::SMEM, s>>>(mq, mk, mv, a);
-  return cudaGetLastError() == cudaSuccess ? FP_OK : FP_ERR_CUDA;
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_last_error("attention launch", (int)e, cudaGetErrorString(e));
+    return FP_ERR_CUDA;
+  }
+  return FP_OK;
 }
 
 }  // namespace

@@ -72,4 +72,7 @@ fp_status_t launch_attention(const Geometry& g, const void* q, const void* k, co
 
 size_t score_smem_bytes(const Geometry& g);
 
+// Records the failing step of the calling thread's last FP_ERR_CUDA (read by fp_last_error).
+void set_last_error(const char* step, int code, const char* detail);
+
 }  // namespace fp

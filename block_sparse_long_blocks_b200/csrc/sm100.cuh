@@ -27,6 +27,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // Every pipeline wait gives up after this long (a healthy wait lasts microseconds).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
+// Per-warpgroup register limit changes (all four warps of the warpgroup execute them).
+template <uint32_t N>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------

@@ -167,6 +167,10 @@ fp_status_t fp_paged_sparse_prefill(const fp_params_t* p, const void* q, const v
  */
 fp_status_t fp_get_device_status(uint32_t* bits, void* stream);
 
+/* Description of the CUDA call behind the calling thread's most recent
+ * FP_ERR_CUDA (thread-local, valid until the next failing call; "" if none). */
+const char* fp_last_error(void);
+
 /* Static, human-readable name of a status code. */
 const char* fp_status_string(fp_status_t s);
 
