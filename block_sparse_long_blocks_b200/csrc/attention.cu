@@ -439,56 +439,61 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st16(tO + c * 16, r16);
           }
         }
+        // P = 2^(s*sl2 - m_ref), computed where it is packed.
+        // The row sum is taken over the rounded weights that the PV MMA consumes,
+        // so O / l is an exact convex combination of V rows: a dominant key's
+        // rounding cancels between numerator and denominator.
         float lsum0 = 0.f, lsum1 = 0.f;
-#pragma unroll
-        for (int c = 0; c < BLK; c += 2) {
-          s[c] = fast_exp2(fmaf(s[c], sl2, -m_ref));
-          s[c + 1] = fast_exp2(fmaf(s[c + 1], sl2, -m_ref));
-          lsum0 += s[c];
-          lsum1 += s[c + 1];
-        }
-        const float lsum = lsum0 + lsum1;
-        l += lsum;
         if constexpr (!FP8) {
 #pragma unroll
           for (int c = 0; c < BLK / 64; ++c) {
             uint32_t pk[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              const __nv_bfloat162 b2 = __floats2bfloat162_rn(s[c * 64 + 2 * e], s[c * 64 + 2 * e + 1]);
-              pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(fast_exp2(fmaf(s[c * 64 + 2 * e], sl2, -m_ref)),
+                                                              fast_exp2(fmaf(s[c * 64 + 2 * e + 1], sl2, -m_ref)));
+              const uint32_t u = *reinterpret_cast<const uint32_t*>(&b2);
+              pk[e] = u;
+              lsum0 += __uint_as_float(u << 16);
+              lsum1 += __uint_as_float(u & 0xFFFF0000u);
             }
             tmem_st32(tS + c * 32, pk);
           }
         } else {
           // P = hi + lo, both e4m3: the residual plane keeps the weights' relative
-          // error near 2^-8 instead of e4m3's 2^-4.
-          uint32_t phi[BLK / 4], plo[BLK / 4];
+          // error near 2^-8 instead of e4m3's 2^-4. Planes: hi in columns
+          // [0, BLK/4), lo in [BLK/4, BLK/2); packed 64 values (16 columns) at a time.
 #pragma unroll
-          for (int e = 0; e < BLK / 4; ++e) {
-            uint32_t h32 = 0, l32 = 0;
+          for (int c = 0; c < BLK / 64; ++c) {
+            uint32_t phi[16], plo[16];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const float x0 = s[4 * e + 2 * q], x1 = s[4 * e + 2 * q + 1];
-              const __nv_fp8x2_storage_t h = __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
-              const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(h, __NV_E4M3);
-              const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-              const __nv_fp8x2_storage_t r =
-                  __nv_cvt_float2_to_fp8x2(make_float2(x0 - hf.x, x1 - hf.y), __NV_SATFINITE, __NV_E4M3);
-              h32 |= (uint32_t)h << (16 * q);
-              l32 |= (uint32_t)r << (16 * q);
+            for (int e = 0; e < 16; ++e) {
+              uint32_t h32 = 0, l32 = 0;
+#pragma unroll
+              for (int q = 0; q < 2; ++q) {
+                const float x0 = fast_exp2(fmaf(s[64 * c + 4 * e + 2 * q], sl2, -m_ref));
+                const float x1 = fast_exp2(fmaf(s[64 * c + 4 * e + 2 * q + 1], sl2, -m_ref));
+                const __nv_fp8x2_storage_t h =
+                    __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
+                const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(h, __NV_E4M3);
+                const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+                const __nv_fp8x2_storage_t r =
+                    __nv_cvt_float2_to_fp8x2(make_float2(x0 - hf.x, x1 - hf.y), __NV_SATFINITE, __NV_E4M3);
+                const __half2_raw rr = __nv_cvt_fp8x2_to_halfraw2(r, __NV_E4M3);
+                const float2 rf = __half22float2(*reinterpret_cast<const __half2*>(&rr));
+                lsum0 += hf.x + rf.x;
+                lsum1 += hf.y + rf.y;
+                h32 |= (uint32_t)h << (16 * q);
+                l32 |= (uint32_t)r << (16 * q);
+              }
+              phi[e] = h32;
+              plo[e] = l32;
             }
-            phi[e] = h32;
-            plo[e] = l32;
-          }
-          if constexpr (BLK / 4 == 32) {
-            tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(phi));
-            tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(plo));
-          } else {
-            tmem_st16(tS, phi);
-            tmem_st16(tS + 16, plo);
+            tmem_st16(tS + 16 * c, phi);
+            tmem_st16(tS + BLK / 4 + 16 * c, plo);
           }
         }
+        l += lsum0 + lsum1;
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full + mt);
