@@ -49,6 +49,15 @@ constexpr uint32_t kSoftmaxRegs = 200;
 constexpr uint32_t kControlRegs = 96;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * 168, "register split exceeds the launch");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// On a rescale the reference max is set this far below the new row max. For
+// e4m3 P this places the running max at P = 16 (P stays <= 2^8 = 256 < 448
+// because the threshold still bounds the reference gap at 8) and moves e4m3's
+// subnormal floor 16x further below it, so far fewer small weights underflow;
+// bf16 P has fp32's exponent range and needs no offset.
+template <bool FP8>
+struct MaxOffset {
+  static constexpr float value = FP8 ? 4.0f : 0.0f;
+};
 constexpr int kSmemBudget = 200 * 1024;
 
 // 2^x with the MUFU.EX2 instruction (flush-to-zero, ~2 ulp); 2^-inf = +0.
@@ -422,10 +431,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 1; c < BLK; ++c) mx = fmaxf(mx, s[c]);
         const float m_new = fmaxf(m_ref, mx * sl2);
         const bool need = m_new > m_ref + kRescaleThreshold;
-        const float f = need ? fast_exp2(m_ref - m_new) : 1.f;
+        const float f = need ? fast_exp2(m_ref - (m_new - MaxOffset<FP8>::value)) : 1.f;
         if (need) {
           l *= f;
-          m_ref = m_new;
+          m_ref = m_new - MaxOffset<FP8>::value;
         }
         // TMEM accesses are warp-collective: rescale when any row of the warp needs it
         if (n > 0 && __any_sync(0xffffffffu, need)) {
@@ -440,9 +449,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         // P = 2^(s*sl2 - m_ref), computed where it is packed.
-        // The row sum is taken over the rounded weights that the PV MMA consumes,
-        // so O / l is an exact convex combination of V rows: a dominant key's
-        // rounding cancels between numerator and denominator.
+        // bf16: the row sum is taken over the rounded weights that the PV MMA
+        // consumes, so O / l is an exact convex combination of V rows and a
+        // dominant key's rounding cancels between numerator and denominator.
+        // e4m3: the row sum is over the float32 weights, which also accounts
+        // for the mass of weights below the e4m3 subnormal floor.
         float lsum0 = 0.f, lsum1 = 0.f;
         if constexpr (!FP8) {
 #pragma unroll
@@ -479,10 +490,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hr));
                 const __nv_fp8x2_storage_t r =
                     __nv_cvt_float2_to_fp8x2(make_float2(x0 - hf.x, x1 - hf.y), __NV_SATFINITE, __NV_E4M3);
-                const __half2_raw rr = __nv_cvt_fp8x2_to_halfraw2(r, __NV_E4M3);
-                const float2 rf = __half22float2(*reinterpret_cast<const __half2*>(&rr));
-                lsum0 += hf.x + rf.x;
-                lsum1 += hf.y + rf.y;
+                lsum0 += x0;
+                lsum1 += x1;
                 h32 |= (uint32_t)h << (16 * q);
                 l32 |= (uint32_t)r << (16 * q);
               }

@@ -148,8 +148,11 @@ fp_status_t fp_discover_compact(const fp_params_t* p, const void* q, const void*
  * q, k, v: contiguous or varlen layout (no page table; p->page_table must be
  * NULL). o: device bf16, same layout as q. lse: NULL or device float
  * [hq, R * max_seqlen] (contiguous) / [hq, total_tokens] (varlen), natural-log
- * sum of exponentials of the scaled logits. Rows with cnt = 0 get O = 0 and
- * lse = -inf. Output rows of tokens outside every request are not written.
+ * sum of exponentials of the scaled logits. With bf16 inputs O is normalised
+ * by the sum of the bf16-rounded softmax weights the PV product uses, and lse
+ * is the log of that same sum (within 2^-8 relative of the exact sum). Rows
+ * with cnt = 0 get O = 0 and lse = -inf. Output rows of tokens outside every
+ * request are not written.
  */
 fp_status_t fp_sparse_prefill(const fp_params_t* p, const void* q, const void* k, const void* v,
                               const int32_t* idx, const int32_t* cnt, void* o, float* lse,

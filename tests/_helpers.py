@@ -239,5 +239,7 @@ def check_attention(dev: Device, orc_out: dict, fp8: bool, report: dict | None =
     else:
         assert mx <= BF16_MAX, f"bf16 max abs err {mx}"
         assert mean <= BF16_MEAN, f"bf16 mean abs err {mean}"
-    assert lse_err <= 2e-3, f"lse max abs err {lse_err}"
+    # bf16: lse is the log of the sum of the bf16-rounded weights (<= 2^-8 relative)
+    lse_tol = 2e-3 if fp8 else 5e-3
+    assert lse_err <= lse_tol, f"lse max abs err {lse_err}"
     return mx, mean
