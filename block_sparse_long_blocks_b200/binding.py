@@ -86,6 +86,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "fp_get_device_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), vp]),
         "fp_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "fp_last_error": (ctypes.c_char_p, []),
+        "fp_discover_compact_static": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp]),
+        "fp_static_scratch_bytes": (sz, []),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -214,6 +216,14 @@ def fp_discover_compact(p: Params, q, k, mask, idx, cnt, workspace, stream=None)
            lib.fp_discover_compact(ctypes.byref(p), q.data_ptr(), k.data_ptr(), _ptr(mask), idx.data_ptr(),
                                    cnt.data_ptr(), workspace.data_ptr(),
                                    workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def fp_discover_compact_static(p: Params, q, k, mask, idx, cnt, stream=None):
+    """fp_discover_compact with the library's fixed scratch array (no workspace)."""
+    lib = load()
+    _check("fp_discover_compact_static",
+           lib.fp_discover_compact_static(ctypes.byref(p), q.data_ptr(), k.data_ptr(), _ptr(mask), idx.data_ptr(),
+                                          cnt.data_ptr(), _stream(stream)))
 
 
 def fp_sparse_prefill(p: Params, q, k, v, idx, cnt, o, lse=None, stream=None):

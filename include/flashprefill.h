@@ -164,6 +164,32 @@ fp_status_t fp_paged_sparse_prefill(const fp_params_t* p, const void* q, const v
                                     void* o, float* lse, void* stream);
 
 /*
+ * Discovery and compaction without a caller-provided workspace: the same
+ * kernels and outputs as fp_discover_compact, with the pooled-Q/K scratch
+ * taken from a fixed device array inside the library. The paper has no
+ * counterpart; this exists for callers that cannot allocate device memory,
+ * such as a plugin inside a host engine that owns all device memory and
+ * exposes no allocator, or a path that must not call cudaMalloc because it
+ * can synchronise the device. It allocates nothing.
+ * - Limit: fp_workspace_size(p) must not exceed fp_static_scratch_bytes()
+ *   (32 MiB, enough for one 128K-token sequence with 32 query / 4 KV heads at
+ *   block 128); larger problems return FP_ERR_WORKSPACE before any launch and
+ *   fp_last_error() says how much was needed.
+ * - The array exists on every GPU that loads the library, until exit. The
+ *   first call on a device looks up the array's device address on that
+ *   device (the device must be current); make that first call before any
+ *   stream capture.
+ * - All calls share the one array and it keeps the last call's contents
+ *   (nothing in it needs to start at zero). Calls whose work overlaps on the
+ *   GPU (e.g. on two streams at once) race on it: serialise them.
+ */
+fp_status_t fp_discover_compact_static(const fp_params_t* p, const void* q, const void* k,
+                                       uint32_t* mask, int32_t* idx, int32_t* cnt, void* stream);
+
+/* Size in bytes of the fixed scratch array fp_discover_compact_static uses. */
+size_t fp_static_scratch_bytes(void);
+
+/*
  * Synchronises `stream`, writes the device status bits (FP_DEV_*) of the
  * current device to *bits (may be NULL) and clears them. Returns FP_OK if no
  * bit was set, FP_ERR_DEVICE otherwise, FP_ERR_CUDA on a runtime error.
