@@ -40,6 +40,18 @@ UNIT = "TFLOPS (dense-equivalent)"
 FP8_OVER_BF16 = 2.0  # nominal dense fp8 / bf16 tensor-core ratio (4.5 / 2.25 PFLOP/s)
 
 
+def blas_threads() -> int:
+    """Threads the oracle's numpy BLAS uses (what the CPU baseline actually ran on)."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d["num_threads"] for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -171,6 +183,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-fp8-extra", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="run a shorter sequence of the same workload (profiling small cases)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -189,6 +203,8 @@ def main():
                                 device_id=torch.device("cuda", local))
 
     w = wl.workloads()[args.workload]
+    if args.seq_len:
+        w = wl.small_case(w, args.seq_len)
     if args.impl == "reference":
         if rank == 0:
             run_reference(args, w, world)
@@ -227,7 +243,7 @@ def run_reference(args, w, world):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "seq_len": w.seqlens[0], "hq": w.hq, "hkv": w.hkv, "block": w.block,
                        "alpha": w.alpha, "input_dtype": args.dtype},
-            "cpu_baseline": {"value": val, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                              "sample": f"per step {last['rows']} (KV group, query block) rows of the layer "
                                        f"(discovery + attention) plus full key pooling, extrapolated by work "
                                        f"counts to all {last['N'] * w.hkv} rows / {total_visits} visited blocks"},
@@ -352,7 +368,7 @@ def run_native(args, w, world, rank, local, dist):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         smp = oracle_sample(w, inp_host, args.cpu_budget, max_rows=10_000)
         t = extrapolate(smp, w, visits)
-        line["cpu_baseline"] = {"value": dense / t / 1e12, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+        line["cpu_baseline"] = {"value": dense / t / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"{smp['rows']} (KV group, query block) rows of the layer (discovery + "
                                           f"attention, {smp['wall']:.1f} s) plus full key pooling, extrapolated by "
                                           f"work counts to {smp['N'] * w.hkv} rows / {visits} visited blocks",
