@@ -67,6 +67,20 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// acc_lo += float(low bf16 of u); acc_hi += float(high bf16 of u)
+__device__ __forceinline__ void add_bf16x2(float& acc_lo, float& acc_hi, uint32_t u) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(acc_lo), "+f"(acc_hi)
+      : "r"(u));
+}
+
 struct AttnArgs {
   Geometry g;
   int Tm;       // tokens per M-tile
@@ -406,8 +420,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         vmul = __ldg(g.v_scale + U.kvh);
       }
       float m_ref = -INFINITY, l = 0.f;
+      // Lists are strictly ascending, so only the last visit can be the
+      // diagonal block (the producer validates every entry).
+      const bool last_is_diag = U.count > 0 && __ldg(a.idx + U.lbase + U.count - 1) == U.i;
       for (int n = 0; n < U.count; ++n) {
-        const int j = list_entry(a, U, n);
         ok = mbar_wait(s_full + mt, (uint32_t)(sn & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
         if (!ok) break;
         ++sn;
@@ -421,14 +437,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < BLK; ++c) s[c] = __uint_as_float(sr[c]);
         }
-        if (j == U.i) {  // diagonal block: keys after the query are masked
+        if (last_is_diag && n == U.count - 1) {  // diagonal block: keys after the query are masked
 #pragma unroll
           for (int c = 0; c < BLK; ++c)
             if (c > qtok) s[c] = -INFINITY;
         }
-        float mx = s[0];
+        float mx;
+        {
+          float m0 = fmaxf(s[0], s[1]), m1 = fmaxf(s[2], s[3]), m2 = fmaxf(s[4], s[5]), m3 = fmaxf(s[6], s[7]);
 #pragma unroll
-        for (int c = 1; c < BLK; ++c) mx = fmaxf(mx, s[c]);
+          for (int c = 8; c < BLK; c += 8) {
+            m0 = fmax3(m0, s[c], s[c + 1]);
+            m1 = fmax3(m1, s[c + 2], s[c + 3]);
+            m2 = fmax3(m2, s[c + 4], s[c + 5]);
+            m3 = fmax3(m3, s[c + 6], s[c + 7]);
+          }
+          mx = fmax3(m0, m1, fmaxf(m2, m3));
+        }
         const float m_new = fmaxf(m_ref, mx * sl2);
         const bool need = m_new > m_ref + kRescaleThreshold;
         const float f = need ? fast_exp2(m_ref - (m_new - MaxOffset<FP8>::value)) : 1.f;
@@ -454,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // dominant key's rounding cancels between numerator and denominator.
         // e4m3: the row sum is over the float32 weights, which also accounts
         // for the mass of weights below the e4m3 subnormal floor.
-        float lsum0 = 0.f, lsum1 = 0.f;
+        float lsum0 = 0.f, lsum1 = 0.f, lsum2 = 0.f, lsum3 = 0.f;
         if constexpr (!FP8) {
 #pragma unroll
           for (int c = 0; c < BLK / 64; ++c) {
@@ -465,8 +490,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                               fast_exp2(fmaf(s[c * 64 + 2 * e + 1], sl2, -m_ref)));
               const uint32_t u = *reinterpret_cast<const uint32_t*>(&b2);
               pk[e] = u;
-              lsum0 += __uint_as_float(u << 16);
-              lsum1 += __uint_as_float(u & 0xFFFF0000u);
+              if (e & 1) add_bf16x2(lsum2, lsum3, u);
+              else add_bf16x2(lsum0, lsum1, u);
             }
             tmem_st32(tS + c * 32, pk);
           }
@@ -490,8 +515,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hr));
                 const __nv_fp8x2_storage_t r =
                     __nv_cvt_float2_to_fp8x2(make_float2(x0 - hf.x, x1 - hf.y), __NV_SATFINITE, __NV_E4M3);
-                lsum0 += x0;
-                lsum1 += x1;
+                if (q) {
+                  lsum2 += x0;
+                  lsum3 += x1;
+                } else {
+                  lsum0 += x0;
+                  lsum1 += x1;
+                }
                 h32 |= (uint32_t)h << (16 * q);
                 l32 |= (uint32_t)r << (16 * q);
               }
@@ -502,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st16(tS + BLK / 4 + 16 * c, plo);
           }
         }
-        l += lsum0 + lsum1;
+        l += (lsum0 + lsum1) + (lsum2 + lsum3);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full + mt);
