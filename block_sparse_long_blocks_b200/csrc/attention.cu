@@ -21,7 +21,8 @@
 // Order of MMAs per visit n (ping-pong): PV0(n), S0(n+1), PV1(n), S1(n+1), so
 // one warpgroup's softmax overlaps the other tile's MMAs.
 // Softmax: online, base-2, with the running reference max raised only when the
-// tile max exceeds it by more than 8 (then O and l are rescaled in place).
+// tile max exceeds it by more than a threshold (64 for bf16, 8 for e4m3; then O
+// and l are rescaled in place).
 // Every wait is time-bounded; on expiry the CTA records FP_DEV_TIMEOUT, drains
 // its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -48,7 +49,19 @@ constexpr int kMmaWarp = 9;
 constexpr uint32_t kSoftmaxRegs = 200;
 constexpr uint32_t kControlRegs = 96;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * 168, "register split exceeds the launch");
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// The reference max is raised only when a tile's max exceeds it by more than
+// this (log2 units); P is then at most 2^threshold. e4m3 P must stay below 448.
+// bf16 P, the float32 row sum and the float32 TMEM accumulators have float32's
+// exponent range: with 2^64 per weight, 2^18 keys and |v| < 2^4 every sum stays
+// below 2^86, so a rescale (a TMEM round trip of the O row) is needed only on
+// jumps of the row max by more than 64 (a factor 1.8e19).
+#ifndef FP_RESCALE_LOG2_BF16
+#define FP_RESCALE_LOG2_BF16 64
+#endif
+template <bool FP8>
+struct RescaleThreshold {
+  static constexpr float value = FP8 ? 8.0f : (float)FP_RESCALE_LOG2_BF16;
+};
 // On a rescale the reference max is set this far below the new row max. For
 // e4m3 P this places the running max at P = 16 (P stays <= 2^8 = 256 < 448
 // because the threshold still bounds the reference gap at 8) and moves e4m3's
@@ -65,6 +78,82 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// ---- packed float32x2 arithmetic (one instruction for two lanes' worth of work)
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair of x <= 8 on the FMA pipe, to take load off the MUFU unit.
+// Cody-Waite style range reduction x = j + f: j = round(x) obtained by adding
+// 1.5*2^23 (the float then holds j in its low mantissa bits), f = x - j in
+// [-0.5, 0.5]; 2^f by a degree-3 polynomial whose coefficients were fitted for
+// minimum maximum relative error on [-0.5, 0.5] (7.5e-5, far below the bf16 /
+// e4m3 rounding that follows); 2^j by adding j to the exponent field. Inputs
+// are clamped at -125 so the exponent field stays normal (2^-125 stands in for
+// 0, which is negligible against a row maximum of at least 1).
+__device__ __forceinline__ void exp2_poly2(uint64_t x2, float& y0, float& y1) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  x2 = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t t2 = f2_add(x2, f2_pack(kMagic, kMagic));
+  const uint64_t r2 = f2_add(t2, f2_pack(-kMagic, -kMagic));
+  const uint64_t f2 = f2_fma(r2, f2_pack(-1.f, -1.f), x2);
+  uint64_t p2 = f2_fma(f2_pack(0.05517132207751274f, 0.05517132207751274f), f2,
+                       f2_pack(0.24261054396629333f, 0.24261054396629333f));
+  p2 = f2_fma(p2, f2, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  p2 = f2_fma(p2, f2, f2_pack(0.9999281167984009f, 0.9999281167984009f));
+  float p0, p1, t0, t1;
+  f2_unpack(p2, p0, p1);
+  f2_unpack(t2, t0, t1);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// One pair of softmax weights 2^(s*sl2 - m): packed scale-and-subtract, then
+// every kEmuEvery-th pair on the FMA pipe and the rest on MUFU.EX2.
+// Tuning knobs (compile time): FP_EMU_EVERY = 0 disables the FMA-pipe exp2;
+// FP_PACKED_FMA selects the packed float32x2 scale-and-subtract.
+#ifndef FP_EMU_EVERY
+#define FP_EMU_EVERY 0
+#endif
+#ifndef FP_PACKED_FMA
+#define FP_PACKED_FMA 1
+#endif
+constexpr int kEmuEvery = FP_EMU_EVERY;
+__device__ __forceinline__ bool emulated_pair(int pair) {
+  return kEmuEvery > 0 && (pair % (kEmuEvery > 0 ? kEmuEvery : 1)) == (kEmuEvery > 0 ? kEmuEvery : 1) - 1;
+}
+__device__ __forceinline__ void exp2_pair(float s0, float s1, float sl2, float m_ref, uint64_t sl2x2, uint64_t negm2,
+                                          bool emulate, float& p0, float& p1) {
+  if (emulate) {
+    exp2_poly2(f2_fma(f2_pack(s0, s1), sl2x2, negm2), p0, p1);
+  } else if (FP_PACKED_FMA) {
+    float x0, x1;
+    f2_unpack(f2_fma(f2_pack(s0, s1), sl2x2, negm2), x0, x1);
+    p0 = fast_exp2(x0);
+    p1 = fast_exp2(x1);
+  } else {
+    p0 = fast_exp2(fmaf(s0, sl2, -m_ref));
+    p1 = fast_exp2(fmaf(s1, sl2, -m_ref));
+  }
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -455,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mx = fmax3(m0, m1, fmaxf(m2, m3));
         }
         const float m_new = fmaxf(m_ref, mx * sl2);
-        const bool need = m_new > m_ref + kRescaleThreshold;
+        const bool need = m_new > m_ref + RescaleThreshold<FP8>::value;
         const float f = need ? fast_exp2(m_ref - (m_new - MaxOffset<FP8>::value)) : 1.f;
         if (need) {
           l *= f;
@@ -480,14 +569,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // e4m3: the row sum is over the float32 weights, which also accounts
         // for the mass of weights below the e4m3 subnormal floor.
         float lsum0 = 0.f, lsum1 = 0.f, lsum2 = 0.f, lsum3 = 0.f;
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_ref, -m_ref);
         if constexpr (!FP8) {
 #pragma unroll
           for (int c = 0; c < BLK / 64; ++c) {
             uint32_t pk[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              const __nv_bfloat162 b2 = __floats2bfloat162_rn(fast_exp2(fmaf(s[c * 64 + 2 * e], sl2, -m_ref)),
-                                                              fast_exp2(fmaf(s[c * 64 + 2 * e + 1], sl2, -m_ref)));
+              float p0, p1;
+              exp2_pair(s[c * 64 + 2 * e], s[c * 64 + 2 * e + 1], sl2, m_ref, sl2x2, negm2, emulated_pair(e), p0,
+                        p1);
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
               const uint32_t u = *reinterpret_cast<const uint32_t*>(&b2);
               pk[e] = u;
               if (e & 1) add_bf16x2(lsum2, lsum3, u);
@@ -507,8 +599,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               uint32_t h32 = 0, l32 = 0;
 #pragma unroll
               for (int q = 0; q < 2; ++q) {
-                const float x0 = fast_exp2(fmaf(s[64 * c + 4 * e + 2 * q], sl2, -m_ref));
-                const float x1 = fast_exp2(fmaf(s[64 * c + 4 * e + 2 * q + 1], sl2, -m_ref));
+                float x0, x1;
+                exp2_pair(s[64 * c + 4 * e + 2 * q], s[64 * c + 4 * e + 2 * q + 1], sl2, m_ref, sl2x2, negm2,
+                          emulated_pair(2 * e + q), x0, x1);
                 const __nv_fp8x2_storage_t h =
                     __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
                 const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(h, __NV_E4M3);
