@@ -40,6 +40,25 @@ UNIT = "TFLOPS (dense-equivalent)"
 FP8_OVER_BF16 = 2.0  # nominal dense fp8 / bf16 tensor-core ratio (4.5 / 2.25 PFLOP/s)
 
 
+def recorded_traffic(workload: str, dtype: str):
+    """DRAM bytes per attention launch from the committed ncu record, if it was taken
+    on the current kernel sources (else None)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)
+        h = hashlib.sha256()
+        for src in rec["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != rec["source_sha256"]:
+            return None
+        e = rec["entries"].get(f"{workload}/{dtype}")
+        return None if e is None else e["dram_read_bytes"] + e["dram_write_bytes"]
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def blas_threads() -> int:
     """Threads the oracle's numpy BLAS uses (what the CPU baseline actually ran on)."""
     try:
@@ -350,7 +369,8 @@ def run_native(args, w, world, rank, local, dist):
             "ms_per_layer": ms_step, "discover_compact_ms": disc_ms, "attention_ms": attn_ms,
             "visited_tile_tflops": achieved,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tc, "unit": "TFLOP/s",
-                         "frac": achieved / peak_tc, "traffic": None,
+                         "frac": achieved / peak_tc, "traffic": recorded_traffic(w.name, args.dtype),
+                         "traffic_unit": "bytes per launch (ncu dram read+write)",
                          "kernel": "sparse_attention_kernel",
                          "peak_source": f"{pk['source']} bf16 burst" + (" x2 (nominal fp8/bf16)" if fp8 else "")},
             "discovery_roofline": {"bound": "hbm", "achieved": disc_bytes / (disc_ms * 1e-3) / 1e9,
