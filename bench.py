@@ -189,6 +189,21 @@ def extrapolate(s: dict, w: wl.Workload, total_visits: int) -> float:
     return s["t_kpool"] + disc + attn
 
 
+# ----------------------------------------------------------------------------- multi-rank
+def max_over_ranks(values, dist, device):
+    """Element-wise max of per-rank timings (the job is as slow as its slowest rank)."""
+    if dist is None:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def weak_value(world: int, flops_per_rank: float, ms: float) -> float:
+    """Whole-job throughput in TFLOP/s when every rank processes its own layer."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -335,10 +350,7 @@ def run_native(args, w, world, rank, local, dist):
     ms = start.elapsed_time(end)
     disc_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    if dist is not None:
-        t = torch.tensor([ms, disc_ms, attn_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, disc_ms, attn_ms = t.tolist()
+    ms, disc_ms, attn_ms = max_over_ranks([ms, disc_ms, attn_ms], dist, dev)
     ms_step = ms / args.steps
 
     # work counts from the lists of the last step
@@ -354,7 +366,7 @@ def run_native(args, w, world, rank, local, dist):
     disc_bytes = qk_bytes + 4 * visits + 4 * cnt.numel()
     peak_tc = (pk["fp8"] if (fp8 and pk["fp8"]) else pk["bf16"] * (FP8_OVER_BF16 if fp8 else 1.0))
     achieved = visited_flops / (attn_ms * 1e-3) / 1e12
-    value = world * dense / (ms_step * 1e-3) / 1e12
+    value = weak_value(world, dense, ms_step)
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -428,12 +440,8 @@ def e2e(args, D, inp_host, dev, stream, dense, world, dist):
         one()
     b.record(stream)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / steps
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t.item()
-    return {"value": world * dense / (ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+    ms = max_over_ranks([a.elapsed_time(b) / steps], dist, dev)[0]
+    return {"value": weak_value(world, dense, ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
 
 
