@@ -67,9 +67,12 @@ struct RescaleThreshold {
 // because the threshold still bounds the reference gap at 8) and moves e4m3's
 // subnormal floor 16x further below it, so far fewer small weights underflow;
 // bf16 P has fp32's exponent range and needs no offset.
+#ifndef FP_E4M3_MAX_OFFSET
+#define FP_E4M3_MAX_OFFSET 4
+#endif
 template <bool FP8>
 struct MaxOffset {
-  static constexpr float value = FP8 ? 4.0f : 0.0f;
+  static constexpr float value = FP8 ? (float)FP_E4M3_MAX_OFFSET : 0.0f;
 };
 constexpr int kSmemBudget = 200 * 1024;
 
@@ -154,6 +157,21 @@ __device__ __forceinline__ void exp2_pair(float s0, float s1, float sl2, float m
     p0 = fast_exp2(fmaf(s0, sl2, -m_ref));
     p1 = fast_exp2(fmaf(s1, sl2, -m_ref));
   }
+}
+
+// e4m3 hi/lo planes of a pair (x0 low, x1 high), computed in f16x2: hi =
+// e4m3(x), lo = e4m3(x - hi). The f16 rounding of x (2^-11) is far below the
+// residual's own e4m3 rounding (2^-4 of |x - hi| <= 2^-8 |x|).
+__device__ __forceinline__ void e4m3_split2(float x0, float x1, uint32_t& hi16, uint32_t& lo16) {
+  unsigned short h8, l8;
+  uint32_t xh, hh, r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(xh) : "f"(x1), "f"(x0));
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(h8) : "r"(xh));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hh) : "h"(h8));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(xh), "r"(hh));
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(l8) : "r"(r));
+  hi16 = h8;
+  lo16 = l8;
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -602,12 +620,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float x0, x1;
                 exp2_pair(s[64 * c + 4 * e + 2 * q], s[64 * c + 4 * e + 2 * q + 1], sl2, m_ref, sl2x2, negm2,
                           emulated_pair(2 * e + q), x0, x1);
-                const __nv_fp8x2_storage_t h =
-                    __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
-                const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(h, __NV_E4M3);
-                const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-                const __nv_fp8x2_storage_t r =
-                    __nv_cvt_float2_to_fp8x2(make_float2(x0 - hf.x, x1 - hf.y), __NV_SATFINITE, __NV_E4M3);
+                uint32_t h, r;
+                e4m3_split2(x0, x1, h, r);
                 if (q) {
                   lsum2 += x0;
                   lsum3 += x1;
@@ -615,8 +629,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                   lsum0 += x0;
                   lsum1 += x1;
                 }
-                h32 |= (uint32_t)h << (16 * q);
-                l32 |= (uint32_t)r << (16 * q);
+                h32 |= h << (16 * q);
+                l32 |= r << (16 * q);
               }
               phi[e] = h32;
               plo[e] = l32;
