@@ -25,6 +25,12 @@ namespace {
 
 constexpr int kPoolThreads = 256;
 constexpr int kScoreThreads = 256;
+// Loads in flight per pooling thread. 4 measured best: 8 costs occupancy
+// (registers) and lowers the achieved bandwidth.
+#ifndef FP_POOL_UNROLL
+#define FP_POOL_UNROLL 4
+#endif
+constexpr int kPoolUnroll = FP_POOL_UNROLL;
 
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 v;
@@ -116,16 +122,17 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geometry g, const ui
     return (long long)off + t;
   };
 
+  // kPoolUnroll independent 16-byte loads in flight per thread
   int t = t0 + p;
-  for (; t + 3 * tpi < t1; t += 4 * tpi) {
-    uint4 x[4];
+  for (; t + (kPoolUnroll - 1) * tpi < t1; t += kPoolUnroll * tpi) {
+    uint4 x[kPoolUnroll];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kPoolUnroll; ++u) {
       const long long row = row_of(t + u * tpi);
       x[u] = row >= 0 ? ld_stream(base + row * row_bytes + head_off) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) accumulate<FP8>(acc, x[u]);
+    for (int u = 0; u < kPoolUnroll; ++u) accumulate<FP8>(acc, x[u]);
   }
   for (; t < t1; t += tpi) {
     const long long row = row_of(t);
@@ -197,9 +204,9 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(Geometry g, const 
   }
   __syncthreads();
 
-  // scores s[hh][j] = scale * qbar_hh . kbar_j, j = 0..i; lane owns 4 consecutive j
   const int n = i + 1;
   const float* kb = kbarT + ((long long)rg * 128) * g.Npad;
+  // scores s[hh][j] = scale * qbar_hh . kbar_j, j = 0..i; lane owns 4 consecutive j
   for (int jb = warp * 128; jb < n; jb += 128 * (kScoreThreads / 32)) {
     const int j4 = jb + 4 * lane;
     if (j4 < n) {
