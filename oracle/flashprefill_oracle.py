@@ -66,7 +66,7 @@ import numpy as np
 __all__ = [
     "num_blocks", "forced_blocks", "pool_blocks", "pooled_scores", "head_keep",
     "block_mask", "discover_row", "compact", "attention_rows", "block_sparse_attention",
-    "flashprefill", "gather_pages", "flashprefill_paged", "row_borderline",
+    "flashprefill", "gather_pages", "flashprefill_paged", "flashprefill_chunk", "row_borderline",
 ]
 
 
@@ -250,6 +250,78 @@ def flashprefill_paged(Q, k_pool, v_pool, cu_seqlens, page_table, page_size: int
         out.append(flashprefill(Q[cu[r]:cu[r + 1]], Kr, Vr, B, alpha, sink_tokens,
                                 window_tokens, scale, attention))
     return out
+
+
+def flashprefill_chunk(Qc, K, V, B: int, alpha: float, sink_tokens: int, window_tokens: int,
+                       scale: float | None = None, attention: bool = True):
+    """Prefill of a request's last queries against its whole KV (chunked prefill
+    with a cached prefix): K/V [kv_len, Hkv, d] hold every token of the
+    request, Qc [q_len, Hq, d] the queries of its last q_len tokens, which sit
+    at positions p0 = kv_len - q_len .. kv_len - 1.
+
+    Same steps as ``flashprefill`` on the block grid of the KV positions
+    (blocks start at the request's first token): a query block is pooled over
+    the queries it holds (blocks wholly before p0 hold none and get an empty
+    list), key blocks over their tokens; scores, threshold, union and sink /
+    window forcing as before; each query attends to the keys of its row's kept
+    blocks at positions <= its own. With q_len = kv_len this is ``flashprefill``.
+    Returns dict(qbar (None rows for empty blocks), kbar, mask, lists, cnt, O
+    [q_len, Hq, d], lse [Hq, q_len], p0)."""
+    d = Qc.shape[-1]
+    scale = default_scale(d) if scale is None else scale
+    if not (math.isfinite(alpha) and alpha >= 0):
+        raise ValueError("alpha must be finite and >= 0")
+    kv_len, q_len = K.shape[0], Qc.shape[0]
+    if q_len > kv_len:
+        raise ValueError("more queries than keys")
+    p0 = kv_len - q_len
+    N = num_blocks(kv_len, B)
+    Hq, Hkv = Qc.shape[1], K.shape[1]
+    G = Hq // Hkv
+    Sb, Wb = forced_blocks(sink_tokens, window_tokens, B)
+    kbar = pool_blocks(K, B)
+    mask = np.zeros((Hkv, N, N), dtype=bool)
+    qbar = [None] * N
+    for i in range(N):
+        lo, hi = max(i * B, p0), min((i + 1) * B, kv_len)
+        if lo >= hi:
+            continue
+        qbar[i] = Qc[lo - p0: hi - p0].sum(axis=0, dtype=np.float64) / (hi - lo)
+    # the keep rule per row, with the same steps as block_mask
+    for i in range(N):
+        if qbar[i] is None:
+            continue
+        for g in range(Hkv):
+            keep = np.zeros(i + 1, dtype=bool)
+            for h in range(g * G, (g + 1) * G):
+                s = scale * (kbar[: i + 1, g, :] @ qbar[i][h])
+                keep |= np.exp(s - s.max()) >= alpha
+            j = np.arange(i + 1)
+            keep |= (j < Sb) | (i - j < Wb)
+            mask[g, i, : i + 1] = keep
+    lists, cnt = compact(mask)
+    res = dict(qbar=qbar, kbar=kbar, mask=mask, lists=lists, cnt=cnt, scale=scale, p0=p0)
+    if attention:
+        O = np.zeros((q_len, Hq, d))
+        lse = np.full((Hq, q_len), -np.inf)
+        for g in range(Hkv):
+            for i in range(N):
+                lo, hi = max(i * B, p0), min((i + 1) * B, kv_len)
+                if lo >= hi:
+                    continue
+                rows = np.arange(lo, hi)
+                keys = np.concatenate([np.arange(j * B, min((j + 1) * B, kv_len)) for j in lists[g][i]])
+                allowed = keys[None, :] <= rows[:, None]
+                for h in range(g * G, (g + 1) * G):
+                    logits = scale * (Qc[rows - p0, h] @ K[keys, g].T)
+                    logits = np.where(allowed, logits, -np.inf)
+                    m = logits.max(axis=1, keepdims=True)
+                    e = np.exp(logits - m)
+                    z = e.sum(axis=1, keepdims=True)
+                    O[rows - p0, h] = (e / z) @ V[keys, g]
+                    lse[h, rows - p0] = (m + np.log(z))[:, 0]
+        res["O"], res["lse"] = O, lse
+    return res
 
 
 def row_borderline(qbar, kbar, scale: float, alpha: float, g: int, i: int, rel: float = 1e-5):

@@ -413,3 +413,68 @@ def test_discover_row_agrees_with_block_mask():
         for i in range(12):
             got = oracle.discover_row(r["qbar"][i, 4 * g: 4 * g + 4], r["kbar"][:, g], i, r["scale"], a, Sb, Wb)
             np.testing.assert_array_equal(got, np.flatnonzero(r["mask"][g, i]))
+
+
+# ----------------------------------------------------------------------------- chunked prefill
+def _chunk_case(kv_len, hq=4, hkv=2, d=8, seed=77):
+    Q, K, V = _rand(kv_len, hq, hkv, d, seed, amp=3.0)
+    return Q, K, V
+
+
+def test_chunk_with_all_queries_is_full_prefill():
+    Q, K, V = _chunk_case(70)
+    full = oracle.flashprefill(Q, K, V, 8, 0.2, 8, 16)
+    ch = oracle.flashprefill_chunk(Q, K, V, 8, 0.2, 8, 16)
+    assert _lists(ch) == _lists(full)
+    np.testing.assert_array_equal(ch["O"], full["O"])
+    np.testing.assert_array_equal(ch["lse"], full["lse"])
+
+
+def test_block_aligned_chunk_equals_full_prefill_rows():
+    """With the chunk boundary on a block boundary every query block holds the
+    same queries as in full prefill, so lists and outputs coincide."""
+    kv_len, B, p0 = 90, 8, 40
+    Q, K, V = _chunk_case(kv_len)
+    full = oracle.flashprefill(Q, K, V, B, 0.2, 8, 16)
+    ch = oracle.flashprefill_chunk(Q[p0:], K, V, B, 0.2, 8, 16)
+    for g in range(2):
+        for i in range(p0 // B):
+            assert len(ch["lists"][g][i]) == 0
+        for i in range(p0 // B, len(full["lists"][g])):
+            assert ch["lists"][g][i].tolist() == full["lists"][g][i].tolist()
+    np.testing.assert_allclose(ch["O"], full["O"][p0:], rtol=0, atol=1e-13)
+
+
+def test_chunk_partial_first_block_pools_present_queries():
+    kv_len, B, p0 = 50, 8, 21  # block 2 holds queries at positions 21..23 only
+    Q, K, V = _chunk_case(kv_len)
+    ch = oracle.flashprefill_chunk(Q[p0:], K, V, B, 0.2, 0, 0, attention=False)
+    assert ch["qbar"][0] is None and ch["qbar"][1] is None
+    np.testing.assert_allclose(ch["qbar"][2], Q[21:24].mean(axis=0), atol=1e-15)
+    np.testing.assert_allclose(ch["qbar"][3], Q[24:32].mean(axis=0), atol=1e-15)
+
+
+@pytest.mark.parametrize("kv_len,p0,alpha", [(64, 13, 0.1), (77, 40, 1.0), (40, 39, 0.0), (33, 0, 3.0)])
+def test_chunk_attention_equals_masked_sdpa(kv_len, p0, alpha):
+    B, hq, hkv, d = 8, 4, 2, 8
+    Q, K, V = _chunk_case(kv_len, hq, hkv, d, seed=kv_len + p0)
+    ch = oracle.flashprefill_chunk(Q[p0:], K, V, B, alpha, 8, 8)
+    # token mask: query position t (p0..kv_len-1) sees key k iff block(k) is kept in row block(t) and k <= t
+    t = np.arange(p0, kv_len)
+    kk = np.arange(kv_len)
+    tm = np.stack([ch["mask"][g][t[:, None] // B, kk[None, :] // B] & (kk[None, :] <= t[:, None])
+                   for g in range(hkv)])
+    q = torch.from_numpy(Q[p0:]).permute(1, 0, 2)[None]
+    k = torch.from_numpy(K).permute(1, 0, 2)[None]
+    v = torch.from_numpy(V).permute(1, 0, 2)[None]
+    m = torch.from_numpy(np.repeat(tm, hq // hkv, axis=0))[None]
+    want = F.scaled_dot_product_attention(q, k, v, attn_mask=m, scale=1 / math.sqrt(d), enable_gqa=True)
+    np.testing.assert_allclose(ch["O"], want[0].permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_chunk_rejects_bad_arguments():
+    Q, K, V = _chunk_case(20)
+    with pytest.raises(ValueError):
+        oracle.flashprefill_chunk(Q, K[:10], V[:10], 8, 0.1, 0, 0)
+    with pytest.raises(ValueError):
+        oracle.flashprefill_chunk(Q[5:], K, V, 8, -1.0, 0, 0)
