@@ -57,6 +57,7 @@ class Params(ctypes.Structure):
         ("page_size", ctypes.c_int),
         ("max_pages_per_req", ctypes.c_int),
         ("num_pages", ctypes.c_int),
+        ("kv_lens", ctypes.c_void_p),
     ]
 
 
@@ -138,6 +139,8 @@ def config_for(w, inp, alpha: Optional[float] = None) -> Config:
         return Config(batch=inp.q.shape[0], max_seqlen=inp.q.shape[1], hq=w.hq, hkv=w.hkv, block=w.block,
                       alpha=a, sink_tokens=w.sink_tokens, window_tokens=w.window_tokens, fp8=fp8)
     lens = (inp.cu_seqlens[1:] - inp.cu_seqlens[:-1]).tolist()
+    if getattr(inp, "kv_lens", None) is not None:
+        lens = inp.kv_lens.tolist()
     paged = inp.page_table is not None
     return Config(batch=len(lens), max_seqlen=max(lens), hq=w.hq, hkv=w.hkv, block=w.block, alpha=a,
                   sink_tokens=w.sink_tokens, window_tokens=w.window_tokens, fp8=fp8,
@@ -151,7 +154,7 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 
 
 def make_params(cfg: Config, q_scale=None, k_scale=None, v_scale=None, cu_seqlens=None,
-                page_table=None) -> Params:
+                page_table=None, kv_lens=None) -> Params:
     p = Params()
     p.dtype = FP_E4M3 if cfg.fp8 else FP_BF16
     p.batch, p.max_seqlen, p.hq, p.hkv = cfg.batch, cfg.max_seqlen, cfg.hq, cfg.hkv
@@ -162,6 +165,7 @@ def make_params(cfg: Config, q_scale=None, k_scale=None, v_scale=None, cu_seqlen
     p.total_tokens = cfg.total_tokens
     p.page_table = _ptr(page_table)
     p.page_size, p.max_pages_per_req, p.num_pages = cfg.page_size, cfg.max_pages_per_req, cfg.num_pages
+    p.kv_lens = _ptr(kv_lens)
     return p
 
 

@@ -67,6 +67,10 @@ fp_status_t validate(const fp_params_t* p, bool attention) {
     if (p->total_tokens < 0) return FP_ERR_INVALID_ARG;
     if (!aligned(p->cu_seqlens, 4)) return FP_ERR_ALIGNMENT;
   }
+  if (p->kv_lens) {  // chunked prefill reads the prefix from the paged cache
+    if (!p->page_table || !p->cu_seqlens) return FP_ERR_INVALID_ARG;
+    if (!aligned(p->kv_lens, 4)) return FP_ERR_ALIGNMENT;
+  }
   if (p->page_table) {
     if (!p->cu_seqlens) return FP_ERR_INVALID_ARG;
     const int P = p->page_size;
@@ -100,6 +104,7 @@ Geometry geometry(const fp_params_t* p) {
   g.thr = p->alpha > 0.f ? (float)std::log((double)p->alpha) : -INFINITY;
   g.fp8 = p->dtype == FP_E4M3;
   g.cu = p->cu_seqlens;
+  g.kv_lens = p->kv_lens;
   g.total_tokens = p->total_tokens;
   g.page_table = p->page_table;
   g.page_size = p->page_table ? p->page_size : 0;

@@ -225,7 +225,11 @@ struct Cfg {
 };
 
 struct Unit {
-  int r, kvh, i, pair, off, len, count;
+  int r, kvh, i, pair;
+  int off;    // first query row of the request
+  int len;    // KV length (positions 0..len-1)
+  int p0;     // position of the request's first query
+  int count;
   long long lbase, rowi;
 };
 
@@ -238,10 +242,13 @@ __device__ __forceinline__ bool decode_unit(long long u, const AttnArgs& a, Unit
   rem /= a.nPairs;
   U.kvh = (int)(rem % g.Hkv);
   U.r = (int)(rem / g.Hkv);
-  request_span(g, U.r, U.off, U.len);
-  const int q0 = U.i * g.B;
-  if (q0 >= U.len) return false;
-  if (U.pair * 2 * a.Tm >= U.len - q0) return false;  // both M-tiles past the request's end
+  int qlen;
+  request_spans(g, U.r, U.off, qlen, U.len);
+  U.p0 = U.len - qlen;
+  // query positions of this pair of M-tiles, clipped to the request's queries
+  const int lo = U.i * g.B + U.pair * 2 * a.Tm;
+  const int hi = min(lo + 2 * a.Tm, min((U.i + 1) * g.B, U.len));
+  if (max(lo, U.p0) >= hi) return false;
   U.rowi = row_index(U.r, U.kvh, U.i, g.Hkv, g.Nmax);
   U.lbase = list_row_base(U.r, U.kvh, U.i, g.Hkv, g.Nmax);
   int c = __ldg(a.cnt + U.rowi);
@@ -371,7 +378,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         mbar_arrive_expect_tx(q_full, q_bytes);
         for (int mt = 0; mt < 2; ++mt) {
-          const int t = U.off + U.i * g.B + (U.pair * 2 + mt) * a.Tm;
+          const int t = U.off + U.i * g.B + (U.pair * 2 + mt) * a.Tm - U.p0;  // may precede the request:
+                                                                               // those rows are never stored
 #pragma unroll
           for (int ch = 0; ch < C::DCH; ++ch)
             tma_load_3d(sQ + mt * C::Q_TILE + ch * 128 * 128, &tmQ, q_full, ch * C::CH_ELEMS, U.kvh * g.G, t);
@@ -517,9 +525,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       Unit U;
       if (!decode_unit(u, a, U)) continue;
       const int qtok = (U.pair * 2 + mt) * a.Tm + tt;  // token within the query block
-      const bool valid = row < a.rows && U.i * g.B + qtok < U.len;
+      const int qpos = U.i * g.B + qtok;               // its position in the request
+      const bool valid = row < a.rows && qpos >= U.p0 && qpos < U.len;
       const int h = U.kvh * g.G + hh;
-      const long long orow = (long long)U.off + (long long)U.i * g.B + qtok;
+      const long long orow = (long long)U.off + qpos - U.p0;
       float sl2 = a.scale_log2;
       float vmul = 1.f;
       if (FP8 && row < a.rows) {

@@ -89,11 +89,13 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geometry g, const ui
   const int i = (item / chunks) % g.Nmax;
   const int r = item / (chunks * g.Nmax);
 
-  int off, len;
-  request_span(g, r, off, len);
-  const int t0 = i * g.B;
-  if (t0 >= len) return;
-  const int t1 = min(t0 + g.B, len);
+  int qoff, qlen, kvlen;
+  request_spans(g, r, qoff, qlen, kvlen);
+  const int p0 = kvlen - qlen;  // position of the first query
+  // keys: every token of the block; queries: those at positions >= p0
+  const int t0 = isK ? i * g.B : max(i * g.B, p0);
+  const int t1 = min(i * g.B + g.B, kvlen);
+  if (t0 >= t1) return;
 
   const int vpt = hc * VPH;            // vectors per token row of the chunk
   const int tpi = kPoolThreads / vpt;  // tokens per iteration
@@ -119,7 +121,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geometry g, const ui
       }
       return (long long)pg * g.page_size + (t & (g.page_size - 1));
     }
-    return (long long)off + t;
+    return isK ? (long long)qoff + t : (long long)qoff + t - p0;
   };
 
   // kPoolUnroll independent 16-byte loads in flight per thread
@@ -186,10 +188,10 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(Geometry g, const 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long rowi = row_index(r, kvh, i, g.Hkv, g.Nmax);
 
-  int off, len;
-  request_span(g, r, off, len);
-  const int Nr = (len + g.B - 1) / g.B;
-  if (i >= Nr) {
+  int qoff, qlen, kvlen;
+  request_spans(g, r, qoff, qlen, kvlen);
+  const int Nr = (kvlen + g.B - 1) / g.B;
+  if (i >= Nr || (i + 1) * g.B <= kvlen - qlen) {  // past the end, or no query in the block
     if (mask)
       for (int w = threadIdx.x; w < g.Wmax; w += kScoreThreads) mask[rowi * g.Wmax + w] = 0u;
     if (cnt && threadIdx.x == 0) cnt[rowi] = 0;

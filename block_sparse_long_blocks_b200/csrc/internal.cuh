@@ -22,6 +22,7 @@ struct Geometry {
   float thr;      // ln(alpha) (-inf for alpha == 0)
   int fp8;        // Q/K/V are e4m3
   const int32_t* cu;        // device cu_seqlens or nullptr
+  const int32_t* kv_lens;   // device KV length per request (chunked prefill) or nullptr
   int total_tokens;
   const int32_t* page_table;  // device or nullptr
   int page_size, page_shift, max_pages, num_pages;
@@ -48,6 +49,25 @@ __device__ __forceinline__ void request_span(const Geometry& g, int r, int& off,
   }
   off = a;
   len = b - a;
+}
+
+// Query rows and KV length of request r. The queries are the request's last
+// qlen tokens, at positions kvlen - qlen .. kvlen - 1 (kvlen == qlen unless
+// kv_lens is given); query t of the request sits in row qoff + t - (kvlen - qlen).
+// Inconsistent lengths make the request empty and set FP_DEV_BAD_SEQLENS.
+__device__ __forceinline__ void request_spans(const Geometry& g, int r, int& qoff, int& qlen, int& kvlen) {
+  request_span(g, r, qoff, qlen);
+  kvlen = qlen;
+  if (g.kv_lens != nullptr) {
+    const int kl = __ldg(g.kv_lens + r);
+    if (kl < qlen || kl > g.L) {
+      atomicOr(g.status, FP_DEV_BAD_SEQLENS);
+      qlen = 0;
+      kvlen = 0;
+      return;
+    }
+    kvlen = kl;
+  }
 }
 
 __host__ __device__ __forceinline__ long long list_row_base(int r, int kvh, int i, int Hkv, int Nmax) {

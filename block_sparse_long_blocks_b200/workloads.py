@@ -219,6 +219,7 @@ class Inputs:
     v_pool: Optional[torch.Tensor] = None
     page_table: Optional[torch.Tensor] = None
     plants: list = field(default_factory=list)
+    kv_lens: Optional[torch.Tensor] = None   # chunked prefill: KV length per request
     # fp8 variants (filled by to_fp8)
     q_scale: Optional[torch.Tensor] = None
     k_scale: Optional[torch.Tensor] = None
@@ -264,10 +265,26 @@ def make_inputs(w: Workload, seqlens: Optional[tuple] = None) -> Inputs:
                   plants=plants)
 
 
+def make_chunked_inputs(w: Workload, kv_lens: tuple, q_lens: tuple) -> Inputs:
+    """Chunked prefill with a cached prefix: request r has kv_lens[r] tokens in
+    the paged KV pool and its last q_lens[r] tokens are the queries (packed by
+    cu_seqlens). The tokens are generated exactly as for full prefill."""
+    if len(kv_lens) != len(q_lens) or any(q > k for q, k in zip(q_lens, kv_lens)):
+        raise ValueError("need one q_len <= kv_len per request")
+    full = make_inputs(w.with_(paged=True, page_size=w.page_size or 64), seqlens=tuple(kv_lens))
+    cu = full.cu_seqlens.tolist()
+    q = torch.cat([full.q[cu[r + 1] - q_lens[r]: cu[r + 1]] for r in range(len(kv_lens))])
+    cuq = torch.zeros(len(q_lens) + 1, dtype=torch.int32)
+    cuq[1:] = torch.cumsum(torch.tensor(q_lens, dtype=torch.int64), 0).to(torch.int32)
+    return Inputs(full.workload, q, cu_seqlens=cuq, k_pool=full.k_pool, v_pool=full.v_pool,
+                  page_table=full.page_table, plants=full.plants,
+                  kv_lens=torch.tensor(kv_lens, dtype=torch.int32))
+
+
 def to_fp8(inp: Inputs) -> Inputs:
     """FP8-e4m3 copy of ``inp`` with per-head absmax scales (over the whole sequence or pool)."""
     out = Inputs(inp.workload, None, cu_seqlens=inp.cu_seqlens, page_table=inp.page_table,
-                 plants=inp.plants, dtype="e4m3")
+                 plants=inp.plants, dtype="e4m3", kv_lens=inp.kv_lens)
     out.q, out.q_scale = quantize_e4m3(inp.q)
     if inp.k is not None:
         out.k, out.k_scale = quantize_e4m3(inp.k)

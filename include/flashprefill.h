@@ -38,9 +38,16 @@
  * - Paged KV (page_table != NULL, requires cu_seqlens): K/V live in pools
  *   [num_pages, page_size, Hkv, d]; token t of request r is slot t % page_size
  *   of pool page page_table[r * max_pages_per_req + t / page_size].
+ * - Chunked prefill with a cached prefix (kv_lens != NULL; needs cu_seqlens
+ *   and page_table): request r has kv_lens[r] tokens in the paged KV cache and
+ *   its queries are its LAST q_len_r = cu[r+1] - cu[r] tokens (positions
+ *   p0 = kv_len - q_len .. kv_len - 1; q_len <= kv_len <= max_seqlen). Blocks
+ *   are laid on the KV positions; a query block is pooled over the queries it
+ *   holds, blocks before p0 get empty lists, and each query attends to kept
+ *   keys at positions <= its own. Without kv_lens, kv_len = q_len (full prefill).
  * - Block grid: per request, blocks of B = block tokens start at the request's
- *   first token; N_r = ceil(L_r / B); Nmax = ceil(max_seqlen / B). Query head h
- *   uses KV head h / G with G = Hq / Hkv.
+ *   first token; N_r = ceil(kv_len_r / B); Nmax = ceil(max_seqlen / B). Query
+ *   head h uses KV head h / G with G = Hq / Hkv.
  * - Mask layout (uint32): word w of row (r, g, i) is
  *   mask[((r * Hkv + g) * Nmax + i) * Wmax + w], Wmax = ceil(Nmax / 32); bit b
  *   of word w is key block j = 32 w + b. Only j <= i can be set.
@@ -100,6 +107,7 @@ typedef struct {
   int page_size;              /* paged: tokens per page (power of two, 16..256) */
   int max_pages_per_req;
   int num_pages;              /* paged: pages in each pool */
+  const int32_t* kv_lens;     /* chunked prefill: device int32 [batch] or NULL (see below) */
 } fp_params_t;
 
 /* Bytes of device scratch fp_discover needs (pooled Q and K, float32). */

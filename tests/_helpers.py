@@ -72,7 +72,8 @@ class Device:
         self.cu = up(inp.cu_seqlens)
         self.table = up(inp.page_table)
         self.qs, self.ks, self.vs = up(inp.q_scale), up(inp.k_scale), up(inp.v_scale)
-        self.p = fb.make_params(self.cfg, self.qs, self.ks, self.vs, self.cu, self.table)
+        self.kv_lens = up(getattr(inp, "kv_lens", None))
+        self.p = fb.make_params(self.cfg, self.qs, self.ks, self.vs, self.cu, self.table, self.kv_lens)
         T = inp.q.shape[0] * inp.q.shape[1] if inp.cu_seqlens is None else inp.q.shape[0]
         self.T = T
         self.bufs = fb.Buffers(self.p, lse_rows=T if lse else 0, o_shape=tuple(inp.q.shape), hq=self.cfg.hq)
@@ -243,3 +244,16 @@ def check_attention(dev: Device, orc_out: dict, fp8: bool, report: dict | None =
     lse_tol = 2e-3 if fp8 else 5e-3
     assert lse_err <= lse_tol, f"lse max abs err {lse_err}"
     return mx, mean
+
+
+def chunk_requests(inp: wl.Inputs):
+    """Per request of a chunked input: (queries [q_len, Hq, d], K [kv_len, Hkv, d],
+    V, first query row) as CPU tensors."""
+    cu = inp.cu_seqlens.tolist()
+    P = inp.workload.page_size
+    out = []
+    for r, kv in enumerate(inp.kv_lens.tolist()):
+        t = torch.arange(kv)
+        pages = inp.page_table[r][t // P].long()
+        out.append((inp.q[cu[r]:cu[r + 1]], inp.k_pool[pages, t % P], inp.v_pool[pages, t % P], cu[r]))
+    return out

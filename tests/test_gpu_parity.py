@@ -277,3 +277,88 @@ def test_full_size_128k(fp8):
     rows = _sample_rows(orc, w)
     H.check_attention(dev, H.oracle_attention(w, inp, orc, rows), fp8, rep)
     print("128K attention:", rep)
+
+
+# ----------------------------------------------------------------------------- chunked prefill
+def _chunk_oracle(w, inp):
+    """Oracle result per request of a chunked input (float64 of the exact inputs)."""
+    res = []
+    for r, (qc, k, v, row0) in enumerate(H.chunk_requests(inp)):
+        qs = inp.q_scale
+        Qc = H.f64(qc, qs)
+        K = H.f64(k, inp.k_scale)
+        V = H.f64(v, inp.v_scale)
+        res.append((oracle.flashprefill_chunk(Qc, K, V, w.block, w.alpha, w.sink_tokens, w.window_tokens), row0))
+    return res
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_chunked_prefill_matches_oracle(fp8):
+    w = W["paged_varlen"]
+    kv = (1500, 700, 2049, 640, 300)
+    ql = (300, 700, 1000, 1, 173)  # ragged first query block, full, one query, ...
+    inp = wl.make_chunked_inputs(w, kv, ql)
+    if fp8:
+        inp = wl.to_fp8(inp)
+    dev = H.Device(w, inp)
+    dev.discover()
+    assert dev.status() == 0
+    orc = _chunk_oracle(w, inp)
+    gl = dev.lists()
+    border = 0
+    for r, (o, _) in enumerate(orc):
+        N = o["mask"].shape[1]
+        for g in range(w.hkv):
+            for i in range(dev.cfg.nmax):
+                want = o["lists"][g][i].tolist() if i < N else []
+                if gl[r][g][i] != want:
+                    qb = np.stack([x if x is not None else np.zeros_like(o["kbar"][0, :1].repeat(w.hq, 0))
+                                   for x in o["qbar"]])
+                    b = oracle.row_borderline(qb, o["kbar"], o["scale"], w.alpha, g, i, H.BORDER_REL)
+                    assert set(gl[r][g][i]) ^ set(want) <= b, (r, g, i)
+                    border += 1
+    dev.attend()
+    assert dev.status() == 0
+    O = dev.bufs.o.double().cpu().numpy()
+    L = dev.bufs.lse.double().cpu().numpy()
+    errs, tot, n, lse_err = [], 0.0, 0, 0.0
+    for o, row0 in orc:
+        q_len = o["O"].shape[0]
+        e = np.abs(O[row0: row0 + q_len] - o["O"])
+        errs.append(e.max())
+        tot += e.sum()
+        n += e.size
+        lse_err = max(lse_err, float(np.abs(L[:, row0: row0 + q_len] - o["lse"]).max()))
+    mx, mean = max(errs), tot / n
+    print("chunked", "fp8" if fp8 else "bf16", dict(max_abs=mx, mean_abs=mean, lse=lse_err, borderline_rows=border))
+    if fp8:
+        assert mx <= H.FP8_MAX
+    else:
+        assert mx <= H.BF16_MAX and mean <= H.BF16_MEAN
+    assert lse_err <= (2e-3 if fp8 else 5e-3)
+
+
+def test_block_aligned_chunk_equals_full_prefill_on_gpu():
+    """A chunk that starts on a block boundary sees the same pooled blocks as full
+    prefill, so its lists and outputs are bit-identical to full prefill's."""
+    w = W["paged_varlen"]
+    kv, q = (1024, 1536), (512, 768)
+    full = wl.make_inputs(w.with_(seqlens=kv))
+    df = H.Device(w, full)
+    df.discover()
+    df.attend()
+    ch = wl.make_chunked_inputs(w, kv, q)
+    dc = H.Device(w, ch)
+    dc.discover()
+    dc.attend()
+    assert dc.status() == 0
+    lf, lc = df.lists(), dc.lists()
+    for r in range(2):
+        p0 = kv[r] - q[r]
+        for g in range(w.hkv):
+            for i in range(p0 // w.block, kv[r] // w.block):
+                assert lc[r][g][i] == lf[r][g][i]
+    cf = full.cu_seqlens.tolist()
+    cc = ch.cu_seqlens.tolist()
+    for r in range(2):
+        assert torch.equal(dc.bufs.o[cc[r]:cc[r + 1]], df.bufs.o[cf[r + 1] - q[r]:cf[r + 1]])

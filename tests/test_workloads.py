@@ -58,3 +58,14 @@ def test_fp8_quantisation_bounds():
     # the per-head absmax lands exactly on the e4m3 maximum
     amax = x.abs().amax(dim=(0, 1, 3))
     assert torch.all(amax == 448)
+
+
+def test_chunked_inputs_take_the_last_tokens_as_queries():
+    w = wl.workloads()["paged_varlen"]
+    ch = wl.make_chunked_inputs(w, kv_lens=(300, 200), q_lens=(100, 200))
+    full = wl.make_inputs(w.with_(seqlens=(300, 200)))
+    assert ch.cu_seqlens.tolist() == [0, 100, 300]
+    assert ch.kv_lens.tolist() == [300, 200]
+    assert torch.equal(ch.q[:100], full.q[200:300])
+    assert torch.equal(ch.q[100:], full.q[300:500])
+    assert torch.equal(ch.k_pool, full.k_pool) and torch.equal(ch.page_table, full.page_table)
