@@ -216,6 +216,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-fp8-extra", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the 256K / paged / chunked measurements")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--seq-len", type=int, default=0,
                     help="run a shorter sequence of the same workload (profiling small cases)")
@@ -298,13 +299,13 @@ def run_native(args, w, world, rank, local, dist):
         inp_host = wl.to_fp8(inp_host)
 
     def setup(inp):
-        cfg = fb.config_for(w, inp)
+        cfg = fb.config_for(inp.workload, inp)
         t = lambda x: None if x is None else x.to(dev).contiguous()  # noqa: E731
         paged = inp.page_table is not None
         d = dict(q=t(inp.q), k=t(inp.k if not paged else inp.k_pool), v=t(inp.v if not paged else inp.v_pool),
                  cu=t(inp.cu_seqlens), table=t(inp.page_table), qs=t(inp.q_scale), ks=t(inp.k_scale),
-                 vs=t(inp.v_scale), paged=paged, cfg=cfg)
-        d["p"] = fb.make_params(cfg, d["qs"], d["ks"], d["vs"], d["cu"], d["table"])
+                 vs=t(inp.v_scale), kv=t(getattr(inp, "kv_lens", None)), paged=paged, cfg=cfg)
+        d["p"] = fb.make_params(cfg, d["qs"], d["ks"], d["vs"], d["cu"], d["table"], d["kv"])
         d["bufs"] = fb.Buffers(d["p"], device=dev, o_shape=tuple(inp.q.shape))
         return d
 
@@ -397,6 +398,10 @@ def run_native(args, w, world, rank, local, dist):
         line["e2e"] = e2e(args, D, inp_host, dev, stream, dense, world, dist)
     if fp8 is False and not args.no_fp8_extra:
         line["fp8"] = fp8_extra(args, w, inp_host, dev, stream, pk, setup, dist)
+    if not args.no_extras:
+        del D
+        torch.cuda.empty_cache()
+        line["other_workloads"] = extra_workloads(args, setup, stream, pk, fp8)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         smp = oracle_sample(w, inp_host, args.cpu_budget, max_rows=10_000)
         t = extrapolate(smp, w, visits)
@@ -406,6 +411,65 @@ def run_native(args, w, world, rank, local, dist):
                                           f"work counts to {smp['N'] * w.hkv} rows / {visits} visited blocks",
                                 "extrapolated_s_per_layer": t}
     return line
+
+
+def chunk_dense_flops(w, kv_lens, q_lens) -> float:
+    """Dense causal attention flops of queries at positions kv-q..kv-1 over keys <= position."""
+    tot = 0.0
+    for kv, q in zip(kv_lens, q_lens):
+        p0 = kv - q
+        tot += (kv * (kv + 1) - p0 * (p0 + 1)) / 2
+    return 4.0 * w.head_dim * w.hq * tot
+
+
+def extra_workloads(args, setup, stream, pk, fp8):
+    """Per-layer time of the other workload shapes (the 256K extreme-sparsity
+    case, the paged/varlen batch and a chunked prefill over the same batch)."""
+    from block_sparse_long_blocks_b200 import binding as fb
+    W = wl.workloads()
+    pv = W["paged_varlen"]
+    kv = pv.seqlens
+    ql = tuple(max(1, L // 4) for L in kv)
+    cases = [("extreme_256k", W["extreme_256k"], lambda: wl.make_inputs(W["extreme_256k"]), None),
+             ("paged_varlen", pv, lambda: wl.make_inputs(pv), None),
+             ("chunked_prefill_last_quarter", pv, lambda: wl.make_chunked_inputs(pv, kv, ql),
+              chunk_dense_flops(pv, kv, ql))]
+    out = {}
+    for name, w, make, dense in cases:
+        inp = make()
+        if fp8:
+            inp = wl.to_fp8(inp)
+        D = setup(inp)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        disc, attn, tot = [], [], []
+        for s in range(3 + 5):
+            ev[0].record(stream)
+            fb.fp_discover_compact(D["p"], D["q"], D["k"], None, D["bufs"].idx, D["bufs"].cnt, D["bufs"].workspace)
+            ev[1].record(stream)
+            if D["paged"]:
+                fb.fp_paged_sparse_prefill(D["p"], D["q"], D["k"], D["v"], D["bufs"].idx, D["bufs"].cnt, D["bufs"].o)
+            else:
+                fb.fp_sparse_prefill(D["p"], D["q"], D["k"], D["v"], D["bufs"].idx, D["bufs"].cnt, D["bufs"].o)
+            ev[2].record(stream)
+            torch.cuda.synchronize()
+            if s >= 3:
+                disc.append(ev[0].elapsed_time(ev[1]))
+                attn.append(ev[1].elapsed_time(ev[2]))
+                tot.append(ev[0].elapsed_time(ev[2]))
+        cnt = D["bufs"].cnt.long()
+        visits = int(cnt.sum().item())
+        flops = visits * 4.0 * w.block * w.block * w.head_dim * w.group
+        a = statistics.mean(attn)
+        t = statistics.mean(tot)
+        dense = w.dense_equiv_flops() if dense is None else dense
+        peak = (pk["fp8"] or pk["bf16"] * FP8_OVER_BF16) if fp8 else pk["bf16"]
+        out[name] = {"ms_per_layer": t, "discover_compact_ms": statistics.mean(disc), "attention_ms": a,
+                     "dense_equiv_tflops": dense / (t * 1e-3) / 1e12,
+                     "visited_tile_tflops": flops / (a * 1e-3) / 1e12, "frac_of_peak": flops / (a * 1e-3) / 1e12 / peak,
+                     "visited_blocks": visits, "tokens": int(inp.q.shape[0] * (inp.q.shape[1] if inp.q.dim() == 4 else 1))}
+        del D, inp
+        torch.cuda.empty_cache()
+    return out
 
 
 def e2e(args, D, inp_host, dev, stream, dense, world, dist):
