@@ -65,7 +65,7 @@ import numpy as np
 
 __all__ = [
     "num_blocks", "forced_blocks", "pool_blocks", "pooled_scores", "head_keep",
-    "block_mask", "discover_row", "compact", "attention_rows", "block_sparse_attention",
+    "block_mask", "head_masks", "per_head_attention", "discover_row", "compact", "attention_rows", "block_sparse_attention",
     "flashprefill", "gather_pages", "flashprefill_paged", "flashprefill_chunk", "row_borderline",
 ]
 
@@ -133,6 +133,44 @@ def block_mask(qbar, kbar, scale: float, alpha: float, Sb: int, Wb: int) -> np.n
     forced = (j <= i) & ((j < Sb) | (i - j < Wb))
     mask |= forced[None]
     return mask
+
+
+def head_masks(qbar, kbar, scale: float, alpha: float, Sb: int, Wb: int) -> np.ndarray:
+    """Per-query-head selection (the per-head reading of the threshold under
+    PackGQA): keep[h, i, j] = head h's own threshold (against its own row max)
+    or j a sink / window block; False above the diagonal. The group mask of
+    ``block_mask`` is the OR of these over the group's heads."""
+    if not (math.isfinite(alpha) and alpha >= 0):
+        raise ValueError("alpha must be finite and >= 0")
+    N, Hq, _ = qbar.shape
+    s = pooled_scores(qbar, kbar, scale)
+    i = np.arange(N)[:, None]
+    j = np.arange(N)[None, :]
+    forced = (j <= i) & ((j < Sb) | (i - j < Wb))
+    keep = np.zeros((Hq, N, N), dtype=bool)
+    for h in range(Hq):
+        keep[h] = head_keep(s[h], alpha) | forced
+    return keep
+
+
+def per_head_attention(Q, K, V, keep, B: int, scale: float):
+    """Attention in which query head h sees only the blocks of its own selection
+    keep[h] (keys <= query). Returns O [L, Hq, d], lse [Hq, L]."""
+    L, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    G = Hq // Hkv
+    N = num_blocks(L, B)
+    O = np.empty((L, Hq, d), dtype=np.float64)
+    lse = np.empty((Hq, L), dtype=np.float64)
+    for h in range(Hq):
+        g = h // G
+        for i in range(N):
+            blocks = [j for j in range(i + 1) if keep[h, i, j]]
+            (o, l), = attention_rows(Q, K, V, g, i, blocks, B, scale, heads=[h]).values()
+            lo, hi = i * B, min((i + 1) * B, L)
+            O[lo:hi, h] = o
+            lse[h, lo:hi] = l
+    return O, lse
 
 
 def discover_row(qbar_i: np.ndarray, kbar_g: np.ndarray, i: int, scale: float, alpha: float,

@@ -478,3 +478,36 @@ def test_chunk_rejects_bad_arguments():
         oracle.flashprefill_chunk(Q, K[:10], V[:10], 8, 0.1, 0, 0)
     with pytest.raises(ValueError):
         oracle.flashprefill_chunk(Q[5:], K, V, 8, -1.0, 0, 0)
+
+
+# ----------------------------------------------------------------------------- per-head masks
+def test_head_masks_union_is_group_mask_and_single_head_group_agrees():
+    Q, K, V = _rand(96, 8, 2, 8, 5, amp=3.0)
+    r = oracle.flashprefill(Q, K, V, 8, 0.2, 8, 16, attention=False)
+    Sb, Wb = oracle.forced_blocks(8, 16, 8)
+    hm = oracle.head_masks(r["qbar"], r["kbar"], r["scale"], 0.2, Sb, Wb)
+    for g in range(2):
+        np.testing.assert_array_equal(hm[4 * g: 4 * g + 4].any(axis=0), r["mask"][g])
+    # with one query head per group the per-head and group selections coincide
+    Q1, K1, V1 = _rand(64, 2, 2, 8, 6, amp=3.0)
+    r1 = oracle.flashprefill(Q1, K1, V1, 8, 0.2, 8, 8)
+    hm1 = oracle.head_masks(r1["qbar"], r1["kbar"], r1["scale"], 0.2, *oracle.forced_blocks(8, 8, 8))
+    np.testing.assert_array_equal(hm1, r1["mask"])
+    O1, l1 = oracle.per_head_attention(Q1, K1, V1, hm1, 8, r1["scale"])
+    np.testing.assert_allclose(O1, r1["O"], rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("alpha", [0.05, 0.5, 1.0])
+def test_per_head_attention_equals_per_head_masked_sdpa(alpha):
+    L, B, hq, hkv, d = 72, 8, 4, 2, 8
+    Q, K, V = _rand(L, hq, hkv, d, 21, amp=4.0)
+    r = oracle.flashprefill(Q, K, V, B, alpha, 8, 8, attention=False)
+    hm = oracle.head_masks(r["qbar"], r["kbar"], r["scale"], alpha, *oracle.forced_blocks(8, 8, B))
+    O, lse = oracle.per_head_attention(Q, K, V, hm, B, r["scale"])
+    t = np.arange(L)
+    tm = np.stack([hm[h][t[:, None] // B, t[None, :] // B] & (t[None, :] <= t[:, None]) for h in range(hq)])
+    q = torch.from_numpy(Q).permute(1, 0, 2)[None]
+    k = torch.from_numpy(np.repeat(K, hq // hkv, axis=1)).permute(1, 0, 2)[None]
+    v = torch.from_numpy(np.repeat(V, hq // hkv, axis=1)).permute(1, 0, 2)[None]
+    want = F.scaled_dot_product_attention(q, k, v, attn_mask=torch.from_numpy(tm)[None], scale=r["scale"])
+    np.testing.assert_allclose(O, want[0].permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
