@@ -298,7 +298,7 @@ def run_native(args, w, world, rank, local, dist):
     if fp8:
         inp_host = wl.to_fp8(inp_host)
 
-    def setup(inp):
+    def setup(inp, per_head=False):
         cfg = fb.config_for(inp.workload, inp)
         t = lambda x: None if x is None else x.to(dev).contiguous()  # noqa: E731
         paged = inp.page_table is not None
@@ -306,6 +306,9 @@ def run_native(args, w, world, rank, local, dist):
                  cu=t(inp.cu_seqlens), table=t(inp.page_table), qs=t(inp.q_scale), ks=t(inp.k_scale),
                  vs=t(inp.v_scale), kv=t(getattr(inp, "kv_lens", None)), paged=paged, cfg=cfg)
         d["p"] = fb.make_params(cfg, d["qs"], d["ks"], d["vs"], d["cu"], d["table"], d["kv"])
+        if per_head:  # per-query-head selection inside the PackGQA tiles
+            d["hb"] = torch.zeros(fb.sizes(d["p"])["list_capacity"], dtype=torch.uint8, device=dev)
+            d["p"] = fb.make_params(cfg, d["qs"], d["ks"], d["vs"], d["cu"], d["table"], d["kv"], d["hb"])
         d["bufs"] = fb.Buffers(d["p"], device=dev, o_shape=tuple(inp.q.shape))
         return d
 
@@ -430,7 +433,9 @@ def extra_workloads(args, setup, stream, pk, fp8):
     pv = W["paged_varlen"]
     kv = pv.seqlens
     ql = tuple(max(1, L // 4) for L in kv)
-    cases = [("extreme_256k", W["extreme_256k"], lambda: wl.make_inputs(W["extreme_256k"]), None),
+    cases = [("qwen30b_128k_per_head_selection", W["qwen30b_128k"], lambda: wl.make_inputs(W["qwen30b_128k"]),
+              None),
+             ("extreme_256k", W["extreme_256k"], lambda: wl.make_inputs(W["extreme_256k"]), None),
              ("paged_varlen", pv, lambda: wl.make_inputs(pv), None),
              ("chunked_prefill_last_quarter", pv, lambda: wl.make_chunked_inputs(pv, kv, ql),
               chunk_dense_flops(pv, kv, ql))]
@@ -439,7 +444,7 @@ def extra_workloads(args, setup, stream, pk, fp8):
         inp = make()
         if fp8:
             inp = wl.to_fp8(inp)
-        D = setup(inp)
+        D = setup(inp, per_head=name.endswith("per_head_selection"))
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         disc, attn, tot = [], [], []
         for s in range(3 + 5):

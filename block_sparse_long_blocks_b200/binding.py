@@ -58,6 +58,7 @@ class Params(ctypes.Structure):
         ("max_pages_per_req", ctypes.c_int),
         ("num_pages", ctypes.c_int),
         ("kv_lens", ctypes.c_void_p),
+        ("head_bits", ctypes.c_void_p),
     ]
 
 
@@ -154,7 +155,7 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 
 
 def make_params(cfg: Config, q_scale=None, k_scale=None, v_scale=None, cu_seqlens=None,
-                page_table=None, kv_lens=None) -> Params:
+                page_table=None, kv_lens=None, head_bits=None) -> Params:
     p = Params()
     p.dtype = FP_E4M3 if cfg.fp8 else FP_BF16
     p.batch, p.max_seqlen, p.hq, p.hkv = cfg.batch, cfg.max_seqlen, cfg.hq, cfg.hkv
@@ -166,6 +167,7 @@ def make_params(cfg: Config, q_scale=None, k_scale=None, v_scale=None, cu_seqlen
     p.page_table = _ptr(page_table)
     p.page_size, p.max_pages_per_req, p.num_pages = cfg.page_size, cfg.max_pages_per_req, cfg.num_pages
     p.kv_lens = _ptr(kv_lens)
+    p.head_bits = _ptr(head_bits)
     return p
 
 

@@ -67,6 +67,7 @@ fp_status_t validate(const fp_params_t* p, bool attention) {
     if (p->total_tokens < 0) return FP_ERR_INVALID_ARG;
     if (!aligned(p->cu_seqlens, 4)) return FP_ERR_ALIGNMENT;
   }
+  if (p->head_bits && G > 8) return FP_ERR_UNSUPPORTED;  // one byte of head bits per list entry
   if (p->kv_lens) {  // chunked prefill reads the prefix from the paged cache
     if (!p->page_table || !p->cu_seqlens) return FP_ERR_INVALID_ARG;
     if (!aligned(p->kv_lens, 4)) return FP_ERR_ALIGNMENT;
@@ -115,6 +116,7 @@ Geometry geometry(const fp_params_t* p) {
   g.q_scale = p->q_scale;
   g.k_scale = p->k_scale;
   g.v_scale = p->v_scale;
+  g.head_bits = p->head_bits;
   g.status = nullptr;
   return g;
 }
@@ -127,6 +129,7 @@ fp_status_t discover_impl(const fp_params_t* p, const void* q, const void* k, ui
   fp_status_t st = validate(p, false);
   if (st != FP_OK) return st;
   if (!q || !k || (!mask && !idx) || (idx && !cnt)) return FP_ERR_INVALID_ARG;
+  if (p->head_bits && !idx) return FP_ERR_INVALID_ARG;  // head bits follow the compacted lists
   if (!aligned(q, 16) || !aligned(k, 16) || (mask && !aligned(mask, 4)) || (idx && !aligned(idx, 4)) ||
       (cnt && !aligned(cnt, 4)))
     return FP_ERR_ALIGNMENT;
@@ -207,6 +210,7 @@ fp_status_t fp_compact(const fp_params_t* p, const uint32_t* mask, int32_t* idx,
   fp_status_t st = validate(p, false);
   if (st != FP_OK) return st;
   if (!mask || !idx || !cnt) return FP_ERR_INVALID_ARG;
+  if (p->head_bits) return FP_ERR_INVALID_ARG;  // the mask holds the group union only
   if (!aligned(mask, 4) || !aligned(idx, 4) || !aligned(cnt, 4)) return FP_ERR_ALIGNMENT;
   Geometry g = geometry(p);
   g.status = status_ptr();

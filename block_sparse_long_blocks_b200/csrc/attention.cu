@@ -154,8 +154,8 @@ __device__ __forceinline__ void exp2_pair(float s0, float s1, float sl2, float m
     p0 = fast_exp2(x0);
     p1 = fast_exp2(x1);
   } else {
-    p0 = fast_exp2(fmaf(s0, sl2, -m_ref));
-    p1 = fast_exp2(fmaf(s1, sl2, -m_ref));
+    p0 = fast_exp2(fmaf(s0, sl2, m_ref == -INFINITY ? 0.f : -m_ref));
+    p1 = fast_exp2(fmaf(s1, sl2, m_ref == -INFINITY ? 0.f : -m_ref));
   }
 }
 
@@ -539,7 +539,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Lists are strictly ascending, so only the last visit can be the
       // diagonal block (the producer validates every entry).
       const bool last_is_diag = U.count > 0 && __ldg(a.idx + U.lbase + U.count - 1) == U.i;
+      // per-head selection: a visited block this row's head did not keep is masked
+      const uint8_t* hbp = g.head_bits ? g.head_bits + U.lbase : nullptr;
+      uint32_t hb_next = (hbp && U.count > 0) ? __ldg(hbp) : 0xFFu;
       for (int n = 0; n < U.count; ++n) {
+        const uint32_t hb = hb_next;
+        if (hbp && n + 1 < U.count) hb_next = __ldg(hbp + n + 1);  // one visit ahead
         ok = mbar_wait(s_full + mt, (uint32_t)(sn & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
         if (!ok) break;
         ++sn;
@@ -557,6 +562,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < BLK; ++c)
             if (c > qtok) s[c] = -INFINITY;
+        }
+        if (!((hb >> hh) & 1u)) {
+#pragma unroll
+          for (int c = 0; c < BLK; ++c) s[c] = -INFINITY;
         }
         float mx;
         {
@@ -596,7 +605,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // e4m3: the row sum is over the float32 weights, which also accounts
         // for the mass of weights below the e4m3 subnormal floor.
         float lsum0 = 0.f, lsum1 = 0.f, lsum2 = 0.f, lsum3 = 0.f;
-        const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_ref, -m_ref);
+        // (m_ref stays -inf while every visited block so far was masked for this row)
+        const float negm = m_ref == -INFINITY ? 0.f : -m_ref;
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(negm, negm);
         if constexpr (!FP8) {
 #pragma unroll
           for (int c = 0; c < BLK / 64; ++c) {
@@ -667,7 +678,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       ++on;
       tc_fence_after();
-      const float inv = vmul / l;
+      const float inv = l > 0.f ? vmul / l : 0.f;  // a row that saw no key (masked everywhere) gets O = 0
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t r32[32];
@@ -686,7 +697,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         }
       }
-      if (valid && a.lse) a.lse[(long long)h * a.T + orow] = (m_ref + log2f(l)) * 0.69314718055994531f;
+      if (valid && a.lse)
+        a.lse[(long long)h * a.T + orow] = l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
       tc_fence_before();
     }
   }

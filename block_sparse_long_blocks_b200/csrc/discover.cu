@@ -178,6 +178,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(Geometry g, const 
   float* qsT = smem;                                           // [128][GP]
   float* sc = qsT + 128 * GP;                                  // [G][Npad]
   uint32_t* words = reinterpret_cast<uint32_t*>(sc + G * g.Npad);  // [Wmax]
+  uint8_t* hbits = reinterpret_cast<uint8_t*>(words + g.Wmax);      // [Npad] per-head bits (optional)
   __shared__ float mx[G];
   __shared__ int warp_tot[kScoreThreads / 32];
 
@@ -257,14 +258,17 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(Geometry g, const 
   __syncthreads();
 
   // keep bits: threshold per head, union over the group, forced sink/window
+  // (a forced block counts as kept by every head of the group)
   for (int w = warp; w < g.Wmax; w += kScoreThreads / 32) {
     const int j = 32 * w + lane;
-    bool keep = false;
+    uint32_t hb = 0;
     if (j < n) {
-      keep = (j < g.Sb) || (i - j < g.Wb);
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh) keep |= (sc[hh * g.Npad + j] - mx[hh] >= g.thr);
+      for (int hh = 0; hh < G; ++hh) hb |= (uint32_t)(sc[hh * g.Npad + j] - mx[hh] >= g.thr) << hh;
+      if ((j < g.Sb) || (i - j < g.Wb)) hb = (1u << G) - 1u;
+      if (g.head_bits) hbits[j] = (uint8_t)hb;
     }
+    const bool keep = hb != 0;
     const uint32_t bits = __ballot_sync(0xffffffffu, keep);
     if (lane == 0) {
       words[w] = bits;
@@ -294,11 +298,15 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(Geometry g, const 
     total += t;
   }
   int pos = before + incl - c;
-  int32_t* dst = idx + list_row_base(r, kvh, i, g.Hkv, g.Nmax);
+  const long long base = list_row_base(r, kvh, i, g.Hkv, g.Nmax);
+  int32_t* dst = idx + base;
+  uint8_t* hdst = g.head_bits ? g.head_bits + base : nullptr;
   uint32_t bits = mine;
   while (bits) {
     const int b = __ffs(bits) - 1;
-    dst[pos++] = 32 * (int)threadIdx.x + b;
+    const int j = 32 * (int)threadIdx.x + b;
+    if (hdst) hdst[pos] = hbits[j];
+    dst[pos++] = j;
     bits &= bits - 1;
   }
   if (threadIdx.x == 0) cnt[rowi] = total;
@@ -367,7 +375,7 @@ cudaError_t launch_score_g(const Geometry& g, const float* qbar, const float* kb
 
 size_t score_smem_bytes(const Geometry& g) {
   const int GP = (g.G + 3) / 4 * 4;
-  return (size_t)(128 * GP + g.G * g.Npad) * sizeof(float) + (size_t)g.Wmax * sizeof(uint32_t);
+  return (size_t)(128 * GP + g.G * g.Npad) * sizeof(float) + (size_t)g.Wmax * sizeof(uint32_t) + (size_t)g.Npad;
 }
 
 cudaError_t launch_pool(const Geometry& g, const void* q, const void* k, float* qbar, float* kbarT,

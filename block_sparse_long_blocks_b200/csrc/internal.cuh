@@ -29,6 +29,7 @@ struct Geometry {
   const float* q_scale;
   const float* k_scale;
   const float* v_scale;
+  uint8_t* head_bits;       // per-head selection bits per list entry, or nullptr
   unsigned* status;         // device status word
 };
 

@@ -45,6 +45,14 @@
  *   are laid on the KV positions; a query block is pooled over the queries it
  *   holds, blocks before p0 get empty lists, and each query attends to kept
  *   keys at positions <= its own. Without kv_lens, kv_len = q_len (full prefill).
+ * - Per-query-head selection (head_bits != NULL; G <= 8): fp_discover_compact
+ *   also writes, for list entry n of row (r, g, i), the byte head_bits[base +
+ *   n] (same offsets as idx) whose bit hh is set iff query head g*G + hh kept
+ *   that block by its own threshold or the block is a sink/window block. The
+ *   attention calls then still visit the group's list (the union, shared K/V
+ *   tiles) but mask, for each query head, the blocks its own bit excludes,
+ *   which gives every head exactly its own selection. fp_compact cannot
+ *   produce the bits (the mask holds the union) and rejects head_bits.
  * - Block grid: per request, blocks of B = block tokens start at the request's
  *   first token; N_r = ceil(kv_len_r / B); Nmax = ceil(max_seqlen / B). Query
  *   head h uses KV head h / G with G = Hq / Hkv.
@@ -108,6 +116,7 @@ typedef struct {
   int max_pages_per_req;
   int num_pages;              /* paged: pages in each pool */
   const int32_t* kv_lens;     /* chunked prefill: device int32 [batch] or NULL (see below) */
+  uint8_t* head_bits;         /* per-head selection: device uint8 [fp_list_capacity(p)] or NULL (see below) */
 } fp_params_t;
 
 /* Bytes of device scratch fp_discover needs (pooled Q and K, float32). */

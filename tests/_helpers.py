@@ -60,7 +60,8 @@ def config_for(w: wl.Workload, inp: wl.Inputs, alpha: float | None = None) -> fb
 class Device:
     """The inputs of one case on the GPU plus the library parameters."""
 
-    def __init__(self, w: wl.Workload, inp: wl.Inputs, alpha: float | None = None, lse: bool = True):
+    def __init__(self, w: wl.Workload, inp: wl.Inputs, alpha: float | None = None, lse: bool = True,
+                 per_head: bool = False):
         self.w, self.inp = w, inp
         self.cfg = config_for(w, inp, alpha)
         dev = "cuda"
@@ -73,7 +74,12 @@ class Device:
         self.table = up(inp.page_table)
         self.qs, self.ks, self.vs = up(inp.q_scale), up(inp.k_scale), up(inp.v_scale)
         self.kv_lens = up(getattr(inp, "kv_lens", None))
-        self.p = fb.make_params(self.cfg, self.qs, self.ks, self.vs, self.cu, self.table, self.kv_lens)
+        self.head_bits = None
+        if per_head:
+            p0 = fb.make_params(self.cfg, self.qs, self.ks, self.vs, self.cu, self.table, self.kv_lens)
+            self.head_bits = torch.zeros(fb.sizes(p0)["list_capacity"], dtype=torch.uint8, device=dev)
+        self.p = fb.make_params(self.cfg, self.qs, self.ks, self.vs, self.cu, self.table, self.kv_lens,
+                                self.head_bits)
         T = inp.q.shape[0] * inp.q.shape[1] if inp.cu_seqlens is None else inp.q.shape[0]
         self.T = T
         self.bufs = fb.Buffers(self.p, lse_rows=T if lse else 0, o_shape=tuple(inp.q.shape), hq=self.cfg.hq)
@@ -256,4 +262,19 @@ def chunk_requests(inp: wl.Inputs):
         t = torch.arange(kv)
         pages = inp.page_table[r][t // P].long()
         out.append((inp.q[cu[r]:cu[r + 1]], inp.k_pool[pages, t % P], inp.v_pool[pages, t % P], cu[r]))
+    return out
+
+
+def head_bits_array(cfg: fb.Config, per_request_lists, per_request_masks, G: int) -> np.ndarray:
+    """Per-head bits in the library's list layout from lists[r][g][i] and the
+    per-head selections keep[r] [Hq, N, N]."""
+    N = cfg.nmax
+    tri = N * (N + 1) // 2
+    out = np.zeros(cfg.batch * cfg.hkv * tri, dtype=np.uint8)
+    for r, (lists, keep) in enumerate(zip(per_request_lists, per_request_masks)):
+        for g, rows in enumerate(lists):
+            for i, l in enumerate(rows):
+                base = (r * cfg.hkv + g) * tri + i * (i + 1) // 2
+                for n, j in enumerate(l):
+                    out[base + n] = sum(int(keep[g * G + hh, i, j]) << hh for hh in range(G))
     return out

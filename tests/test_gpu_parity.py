@@ -362,3 +362,67 @@ def test_block_aligned_chunk_equals_full_prefill_on_gpu():
     cc = ch.cu_seqlens.tolist()
     for r in range(2):
         assert torch.equal(dc.bufs.o[cc[r]:cc[r + 1]], df.bufs.o[cf[r + 1] - q[r]:cf[r + 1]])
+
+
+# ----------------------------------------------------------------------------- per-head selection
+@pytest.mark.parametrize("name,L,fp8", [("qwen30b_128k", 3000, False), ("qwen30b_128k", 3000, True),
+                                        ("tiny2k", None, False)])
+def test_per_head_selection_matches_oracle(name, L, fp8):
+    w = _case(name, L)
+    inp = _inputs(w, fp8)
+    dev = H.Device(w, inp, per_head=True)
+    dev.discover()
+    assert dev.status() == 0
+    orc = H.oracle_discovery(w, inp)
+    H.compare_lists(orc, dev.lists())
+    Sb, Wb = oracle.forced_blocks(w.sink_tokens, w.window_tokens, w.block)
+    keep = [oracle.head_masks(o["qbar"], o["kbar"], o["scale"], w.alpha, Sb, Wb) for o in orc]
+    want = H.head_bits_array(dev.cfg, [o["lists"] for o in orc], keep, w.group)
+    got = dev.head_bits.cpu().numpy()
+    gl = dev.lists()
+    N = dev.cfg.nmax
+    tri = N * (N + 1) // 2
+    for g in range(w.hkv):
+        for i in range(N):
+            base = g * tri + i * (i + 1) // 2
+            if gl[0][g][i] != [int(x) for x in orc[0]["lists"][g][i]]:
+                continue  # borderline rows (already checked by compare_lists)
+            n = len(gl[0][g][i])
+            if not np.array_equal(got[base:base + n], want[base:base + n]):
+                b = oracle.row_borderline(orc[0]["qbar"], orc[0]["kbar"], orc[0]["scale"], w.alpha, g, i,
+                                          H.BORDER_REL)
+                bad = [gl[0][g][i][k] for k in range(n) if got[base + k] != want[base + k]]
+                assert set(bad) <= b, (g, i, bad)
+    # attention on the oracle's lists and head bits against per-head attention
+    idx, cnt = H.upload_lists(dev.cfg, [o["lists"] for o in orc])
+    dev.head_bits.copy_(torch.from_numpy(want))
+    dev.attend(idx, cnt)
+    assert dev.status() == 0
+    q, k, v = H.request_views(inp)[0]
+    O, lse = oracle.per_head_attention(H.f64(q, inp.q_scale), H.f64(k, inp.k_scale), H.f64(v, inp.v_scale),
+                                       keep[0], w.block, oracle.default_scale(w.head_dim))
+    go = dev.bufs.o[0].double().cpu().numpy()
+    e = np.abs(go - O)
+    gl_ = dev.bufs.lse.double().cpu().numpy()
+    print("per-head", name, "fp8" if fp8 else "bf16", dict(max_abs=e.max(), mean_abs=e.mean(),
+                                                             lse=np.abs(gl_ - lse).max()))
+    if fp8:
+        assert e.max() <= H.FP8_MAX
+    else:
+        assert e.max() <= H.BF16_MAX and e.mean() <= H.BF16_MEAN
+    assert np.abs(gl_ - lse).max() <= (2e-3 if fp8 else 5e-3)
+
+
+def test_per_head_with_every_head_selecting_equals_group_mode():
+    """At alpha = 0 every head keeps every causal block: per-head mode must
+    reproduce group (union) mode bit for bit."""
+    w = _case("qwen30b_128k", 1500)
+    inp = _inputs(w)
+    d1 = H.Device(w, inp, 0.0)
+    d1.discover()
+    d1.attend()
+    d2 = H.Device(w, inp, 0.0, per_head=True)
+    d2.discover()
+    d2.attend()
+    assert torch.equal(d1.bufs.cnt, d2.bufs.cnt)
+    assert torch.equal(d1.bufs.o, d2.bufs.o) and torch.equal(d1.bufs.lse, d2.bufs.lse)
