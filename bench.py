@@ -405,6 +405,8 @@ def run_native(args, w, world, rank, local, dist):
         del D
         torch.cuda.empty_cache()
         line["other_workloads"] = extra_workloads(args, setup, stream, pk, fp8)
+        if not fp8:
+            line["other_workloads"]["short_4k"] = short_context(setup, stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         smp = oracle_sample(w, inp_host, args.cpu_budget, max_rows=10_000)
         t = extrapolate(smp, w, visits)
@@ -474,6 +476,52 @@ def extra_workloads(args, setup, stream, pk, fp8):
                      "visited_blocks": visits, "tokens": int(inp.q.shape[0] * (inp.q.shape[1] if inp.q.dim() == 4 else 1))}
         del D, inp
         torch.cuda.empty_cache()
+    return out
+
+
+def short_context(setup, stream):
+    """4K-token prefill (128K workload's shapes and generator): per-layer time of
+    the separate calls, of the single fp_prefill call, and of a CUDA-graph
+    replay of fp_prefill (launch overheads matter at this size)."""
+    from block_sparse_long_blocks_b200 import binding as fb
+    w = wl.small_case(wl.workloads()["qwen30b_128k"], 4096)
+    D = setup(wl.make_inputs(w))
+    b = D["bufs"]
+
+    def separate():
+        fb.fp_discover_compact(D["p"], D["q"], D["k"], None, b.idx, b.cnt, b.workspace)
+        fb.fp_sparse_prefill(D["p"], D["q"], D["k"], D["v"], b.idx, b.cnt, b.o)
+
+    def single():
+        fb.fp_prefill(D["p"], D["q"], D["k"], D["v"], None, b.idx, b.cnt, b.o, b.workspace)
+
+    def timed(fn, n=50):
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    out = {"tokens": 4096, "separate_calls_ms": timed(separate), "fp_prefill_ms": timed(single)}
+    try:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            single()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=side):
+                single()
+        out["fp_prefill_graph_ms"] = timed(g.replay)
+    except RuntimeError as e:  # graph capture unavailable: report, do not fail the bench
+        out["fp_prefill_graph_error"] = str(e)[:200]
+    dense = w.dense_equiv_flops()
+    out["dense_equiv_tflops_fp_prefill"] = dense / (out["fp_prefill_ms"] * 1e-3) / 1e12
     return out
 
 

@@ -89,6 +89,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "fp_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "fp_last_error": (ctypes.c_char_p, []),
         "fp_discover_compact_static": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp]),
+        "fp_prefill": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "fp_static_scratch_bytes": (sz, []),
     }
     for name, (res, args) in sig.items():
@@ -245,6 +246,15 @@ def fp_paged_sparse_prefill(p: Params, q, k_pool, v_pool, idx, cnt, o, lse=None,
            lib.fp_paged_sparse_prefill(ctypes.byref(p), q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
                                        idx.data_ptr(), cnt.data_ptr(), o.data_ptr(), _ptr(lse),
                                        _stream(stream)))
+
+
+def fp_prefill(p: Params, q, k, v, mask, idx, cnt, o, workspace, lse=None, stream=None):
+    """The whole path in one call (discovery + compaction + attention, device work queue)."""
+    lib = load()
+    _check("fp_prefill",
+           lib.fp_prefill(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(mask), idx.data_ptr(),
+                          cnt.data_ptr(), o.data_ptr(), _ptr(lse), workspace.data_ptr(),
+                          workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def fp_get_device_status(stream=None) -> int:

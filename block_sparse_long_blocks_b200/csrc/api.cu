@@ -117,6 +117,7 @@ Geometry geometry(const fp_params_t* p) {
   g.k_scale = p->k_scale;
   g.v_scale = p->v_scale;
   g.head_bits = p->head_bits;
+  g.attn_queue = nullptr;
   g.status = nullptr;
   return g;
 }
@@ -124,8 +125,13 @@ Geometry geometry(const fp_params_t* p) {
 size_t qbar_floats(const Geometry& g) { return (size_t)g.R * g.Nmax * g.Hq * 128; }
 size_t kbar_floats(const Geometry& g) { return (size_t)g.R * g.Hkv * 128 * g.Npad; }
 
+// The attention work-queue counter lives right after the pooled tensors.
+int* queue_slot(const Geometry& g, void* ws) {
+  return reinterpret_cast<int*>(static_cast<float*>(ws) + (qbar_floats(g) + 63) / 64 * 64 + kbar_floats(g));
+}
+
 fp_status_t discover_impl(const fp_params_t* p, const void* q, const void* k, uint32_t* mask, int32_t* idx,
-                          int32_t* cnt, void* ws, size_t ws_bytes, void* stream) {
+                          int32_t* cnt, void* ws, size_t ws_bytes, void* stream, bool zero_queue = false) {
   fp_status_t st = validate(p, false);
   if (st != FP_OK) return st;
   if (!q || !k || (!mask && !idx) || (idx && !cnt)) return FP_ERR_INVALID_ARG;
@@ -138,6 +144,7 @@ fp_status_t discover_impl(const fp_params_t* p, const void* q, const void* k, ui
   if (score_smem_bytes(g) > 227 * 1024) return FP_ERR_UNSUPPORTED;
   g.status = status_ptr();
   if (!g.status) return cuda_fail("device status symbol", cudaGetLastError());
+  if (zero_queue) g.attn_queue = queue_slot(g, ws);
   float* qbar = static_cast<float*>(ws);
   float* kbarT = qbar + (qbar_floats(g) + 63) / 64 * 64;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -160,7 +167,7 @@ fp_status_t attention_impl(const fp_params_t* p, bool paged, const void* q, cons
   Geometry g = geometry(p);
   g.status = status_ptr();
   if (!g.status) return cuda_fail("device status symbol", cudaGetLastError());
-  return launch_attention(g, q, k, v, idx, cnt, o, lse, static_cast<cudaStream_t>(stream));
+  return launch_attention(g, q, k, v, idx, cnt, o, lse, static_cast<cudaStream_t>(stream), nullptr, false);
 }
 
 }  // namespace
@@ -173,7 +180,7 @@ extern "C" {
 size_t fp_workspace_size(const fp_params_t* p) {
   if (validate(p, false) != FP_OK) return 0;
   const Geometry g = geometry(p);
-  return ((qbar_floats(g) + 63) / 64 * 64 + kbar_floats(g)) * sizeof(float);
+  return ((qbar_floats(g) + 63) / 64 * 64 + kbar_floats(g)) * sizeof(float) + 256;  // + work-queue counter
 }
 
 size_t fp_mask_words(const fp_params_t* p) {
@@ -227,6 +234,21 @@ fp_status_t fp_sparse_prefill(const fp_params_t* p, const void* q, const void* k
 fp_status_t fp_paged_sparse_prefill(const fp_params_t* p, const void* q, const void* k_pool, const void* v_pool,
                                     const int32_t* idx, const int32_t* cnt, void* o, float* lse, void* stream) {
   return attention_impl(p, true, q, k_pool, v_pool, idx, cnt, o, lse, stream);
+}
+
+fp_status_t fp_prefill(const fp_params_t* p, const void* q, const void* k, const void* v, uint32_t* mask,
+                       int32_t* idx, int32_t* cnt, void* o, float* lse, void* workspace, size_t ws_bytes,
+                       void* stream) {
+  fp_status_t st = validate(p, true);
+  if (st != FP_OK) return st;
+  if (!v || !o) return FP_ERR_INVALID_ARG;
+  if (!aligned(v, 16) || !aligned(o, 16) || (lse && !aligned(lse, 4))) return FP_ERR_ALIGNMENT;
+  st = discover_impl(p, q, k, mask, idx, cnt, workspace, ws_bytes, stream, /*zero_queue=*/true);
+  if (st != FP_OK) return st;
+  Geometry g = geometry(p);
+  g.status = status_ptr();
+  return launch_attention(g, q, k, v, idx, cnt, o, lse, static_cast<cudaStream_t>(stream), queue_slot(g, workspace),
+                          /*pdl=*/true);
 }
 
 fp_status_t fp_get_device_status(uint32_t* bits, void* stream) {

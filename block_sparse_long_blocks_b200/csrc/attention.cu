@@ -29,6 +29,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include <climits>
 #include <cstdio>
 #include <mutex>
 
@@ -40,6 +41,8 @@ namespace fp {
 namespace {
 
 constexpr int kThreads = 384;  // 3 warpgroups
+constexpr int kUnitRing = 4;                // work units handed from the producer to the other roles
+constexpr int kUnitConsumers = 1 + 256;     // the MMA thread + both softmax warpgroups
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 // Launched at 168 registers/thread (384 x 168 = 64512). The softmax warpgroups
@@ -200,6 +203,7 @@ struct AttnArgs {
   const int32_t* cnt;
   __nv_bfloat16* o;
   float* lse;
+  int* queue;  // device work-queue counter (zeroed before launch) or nullptr: static schedule
 };
 
 template <bool FP8, int BLK>
@@ -216,12 +220,55 @@ struct Cfg {
   static constexpr int QK_STEPS = 128 * ES / KSTEP_BYTES; // 8 (bf16) / 4 (e4m3)
   static constexpr int PV_KEYS = KSTEP_BYTES / ES;        // keys per PV MMA: 16 / 32
   static constexpr int PV_STEPS = BLK / PV_KEYS;
-  static constexpr int NUM_BARS = 2 + 4 * STAGES + 6 + 1;
-  static constexpr int SMEM_USED = 1024 + 2 * Q_TILE + 2 * STAGES * KV_TILE + NUM_BARS * 8 + 16;
+  static constexpr int NUM_BARS = 2 + 4 * STAGES + 6 + 1 + 2 * kUnitRing;
+  static constexpr int SMEM_USED = 1024 + 2 * Q_TILE + 2 * STAGES * KV_TILE + NUM_BARS * 8 + 16 + 4 * kUnitRing;
   // more than half of the SM's shared memory: one CTA per SM, so the CTA's
   // 512-column TMEM allocation never waits for a co-resident CTA
   static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   static_assert(STAGES >= 2, "shared memory budget too small");
+};
+
+// Work units reach the roles either by a static stride over the persistent
+// grid or, with a device queue, in claim order: the producer claims each unit
+// (atomicAdd on the queue) and passes it to the MMA and softmax roles through
+// a small ring in shared memory guarded by full/empty mbarriers.
+struct UnitIter {
+  int* queue;
+  int* ring;
+  uint64_t* full;
+  uint64_t* empty;
+  volatile int* abort;
+  unsigned* status;
+  bool producer;
+  long long u;
+  int n;
+
+  __device__ __forceinline__ long long step(bool first, bool& ok) {
+    if (queue == nullptr) {
+      u = first ? (long long)blockIdx.x : u + gridDim.x;
+      return u;
+    }
+    const int slot = n % kUnitRing;
+    const uint32_t ph = (uint32_t)((n / kUnitRing) & 1);
+    ++n;
+    if (producer) {
+      if (!mbar_wait(empty + slot, ph ^ 1u, abort, status, FP_DEV_TIMEOUT)) {
+        ok = false;
+        return LLONG_MAX;
+      }
+      const int v = atomicAdd(queue, 1);
+      ring[slot] = v;
+      mbar_arrive(full + slot);
+      return v;
+    }
+    if (!mbar_wait(full + slot, ph, abort, status, FP_DEV_TIMEOUT)) {
+      ok = false;
+      return LLONG_MAX;
+    }
+    const int v = ring[slot];
+    mbar_arrive(empty + slot);
+    return v;
+  }
 };
 
 struct Unit {
@@ -319,8 +366,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = s_full + 2;   // [2]
   uint64_t* o_full = p_full + 2;   // [2]
   uint64_t* drain = o_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* unit_full = drain + 1;             // [kUnitRing]
+  uint64_t* unit_empty = unit_full + kUnitRing;  // [kUnitRing]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(unit_empty + kUnitRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* unit_ring = const_cast<int*>(reinterpret_cast<volatile int*>(abort_flag + 1));  // [kUnitRing]
 
   const Geometry& g = a.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -340,6 +390,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(o_full + m, 1);
     }
     mbar_init(drain, 1);
+    for (int k = 0; k < kUnitRing; ++k) {
+      mbar_init(unit_full + k, 1);
+      mbar_init(unit_empty + k, kUnitConsumers);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -361,6 +415,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // With programmatic dependent launch the prologue above overlapped the
+  // previous kernel (discovery); wait for its results before reading lists.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
   if (warp >= 8) reg_dealloc<kControlRegs>();
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ producer
@@ -371,7 +429,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       long long kt = 0, vt = 0, qn = 0;
       const uint32_t q_bytes = 2u * C::DCH * a.rows * 128u;
       bool ok = true;
-      for (long long u = blockIdx.x; u < a.num_units && ok; u += gridDim.x) {
+      UnitIter it{a.queue, unit_ring, unit_full, unit_empty, abort_flag, g.status, true, 0, 0};
+      for (long long u = it.step(true, ok); u < a.num_units && ok; u = it.step(false, ok)) {
         Unit U;
         if (!decode_unit(u, a, U) || U.count == 0) continue;
         ok = mbar_wait(q_empty, (uint32_t)(qn & 1) ^ 1u, abort_flag, g.status, FP_DEV_TIMEOUT);
@@ -450,7 +509,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
 
-      for (long long u = blockIdx.x; u < a.num_units && ok; u += gridDim.x) {
+      UnitIter it{a.queue, unit_ring, unit_full, unit_empty, abort_flag, g.status, false, 0, 0};
+      for (long long u = it.step(true, ok); u < a.num_units && ok; u = it.step(false, ok)) {
         Unit U;
         if (!decode_unit(u, a, U) || U.count == 0) continue;
         ok = mbar_wait(q_full, (uint32_t)(qn & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
@@ -521,7 +581,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int hh = row % g.G, tt = row / g.G;
     long long sn = 0, on = 0;
     bool ok = true;
-    for (long long u = blockIdx.x; u < a.num_units && ok; u += gridDim.x) {
+    UnitIter it{a.queue, unit_ring, unit_full, unit_empty, abort_flag, g.status, false, 0, 0};
+    for (long long u = it.step(true, ok); u < a.num_units && ok; u = it.step(false, ok)) {
       Unit U;
       if (!decode_unit(u, a, U)) continue;
       const int qtok = (U.pair * 2 + mt) * a.Tm + tt;  // token within the query block
@@ -759,7 +820,7 @@ int sm_count() {
 }
 
 template <bool FP8, int BLK, bool PAGED>
-fp_status_t run(const AttnArgs& a, const void* q, const void* k, const void* v, cudaStream_t s) {
+fp_status_t run(const AttnArgs& a, const void* q, const void* k, const void* v, cudaStream_t s, bool pdl) {
   using C = Cfg<FP8, BLK>;
   const Geometry& g = a.g;
   const cuuint64_t es = FP8 ? 1 : 2;
@@ -792,8 +853,18 @@ fp_status_t run(const AttnArgs& a, const void* q, const void* k, const void* v, 
   }
   const long long grid = a.num_units < sm_count() ? a.num_units : sm_count();
   if (grid <= 0) return FP_OK;
-  kern<<<(unsigned)grid, kThreads, C::SMEM, s>>>(mq, mk, mv, a);
-  e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, a);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_last_error("attention launch", (int)e, cudaGetErrorString(e));
     return FP_ERR_CUDA;
@@ -804,13 +875,15 @@ fp_status_t run(const AttnArgs& a, const void* q, const void* k, const void* v, 
 }  // namespace
 
 fp_status_t launch_attention(const Geometry& g, const void* q, const void* k, const void* v, const int32_t* idx,
-                             const int32_t* cnt, void* o, float* lse, cudaStream_t s) {
+                             const int32_t* cnt, void* o, float* lse, cudaStream_t s, int* queue, bool pdl) {
   AttnArgs a;
+  a.queue = queue;
   a.g = g;
   int Tm = 1;
   while (Tm * 2 * g.G <= 128 && Tm * 2 <= g.B) Tm *= 2;
   const int nM = g.B / Tm;
   if (nM < 2 || nM % 2 != 0) return FP_ERR_UNSUPPORTED;
+  if ((long long)g.Nmax * g.R * g.Hkv * (nM / 2) >= INT_MAX) return FP_ERR_UNSUPPORTED;  // int unit ids
   a.Tm = Tm;
   a.rows = Tm * g.G;
   a.nPairs = nM / 2;
@@ -823,12 +896,12 @@ fp_status_t launch_attention(const Geometry& g, const void* q, const void* k, co
   a.lse = lse;
   const bool paged = g.page_table != nullptr;
   if (g.B == 128) {
-    if (g.fp8) return paged ? run<true, 128, true>(a, q, k, v, s) : run<true, 128, false>(a, q, k, v, s);
-    return paged ? run<false, 128, true>(a, q, k, v, s) : run<false, 128, false>(a, q, k, v, s);
+    if (g.fp8) return paged ? run<true, 128, true>(a, q, k, v, s, pdl) : run<true, 128, false>(a, q, k, v, s, pdl);
+    return paged ? run<false, 128, true>(a, q, k, v, s, pdl) : run<false, 128, false>(a, q, k, v, s, pdl);
   }
   if (g.B == 64) {
-    if (g.fp8) return paged ? run<true, 64, true>(a, q, k, v, s) : run<true, 64, false>(a, q, k, v, s);
-    return paged ? run<false, 64, true>(a, q, k, v, s) : run<false, 64, false>(a, q, k, v, s);
+    if (g.fp8) return paged ? run<true, 64, true>(a, q, k, v, s, pdl) : run<true, 64, false>(a, q, k, v, s, pdl);
+    return paged ? run<false, 64, true>(a, q, k, v, s, pdl) : run<false, 64, false>(a, q, k, v, s, pdl);
   }
   return FP_ERR_UNSUPPORTED;
 }

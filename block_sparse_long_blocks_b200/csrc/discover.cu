@@ -182,6 +182,9 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(Geometry g, const 
   __shared__ float mx[G];
   __shared__ int warp_tot[kScoreThreads / 32];
 
+  // a following programmatic-dependent launch (the attention) may start its prologue
+  asm volatile("griddepcontrol.launch_dependents;");
+  if (blockIdx.x == 0 && threadIdx.x == 0 && g.attn_queue) *g.attn_queue = 0;
   const int RH = g.R * g.Hkv;
   const int i = g.Nmax - 1 - (int)(blockIdx.x / RH);
   const int rg = blockIdx.x % RH;

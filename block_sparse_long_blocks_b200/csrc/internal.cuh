@@ -30,6 +30,7 @@ struct Geometry {
   const float* k_scale;
   const float* v_scale;
   uint8_t* head_bits;       // per-head selection bits per list entry, or nullptr
+  int* attn_queue;          // discovery zeroes this attention work-queue counter, or nullptr
   unsigned* status;         // device status word
 };
 
@@ -87,9 +88,11 @@ cudaError_t launch_score(const Geometry& g, const float* qbar, const float* kbar
 cudaError_t launch_compact(const Geometry& g, const uint32_t* mask, int32_t* idx, int32_t* cnt,
                            cudaStream_t s);
 // Returns FP_OK, FP_ERR_UNSUPPORTED or FP_ERR_CUDA.
+// queue: zeroed device counter for claim-order scheduling, or nullptr (static
+// stride). pdl: launch as a programmatic dependent of the previous kernel.
 fp_status_t launch_attention(const Geometry& g, const void* q, const void* k, const void* v,
                              const int32_t* idx, const int32_t* cnt, void* o, float* lse,
-                             cudaStream_t s);
+                             cudaStream_t s, int* queue, bool pdl);
 
 size_t score_smem_bytes(const Geometry& g);
 

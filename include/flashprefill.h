@@ -181,6 +181,21 @@ fp_status_t fp_paged_sparse_prefill(const fp_params_t* p, const void* q, const v
                                     void* o, float* lse, void* stream);
 
 /*
+ * The whole path in one call: discovery + compaction (as fp_discover_compact,
+ * mask may be NULL) followed by the block-sparse attention (as
+ * fp_sparse_prefill, or fp_paged_sparse_prefill when p->page_table is set;
+ * k and v are then the pools). The attention is launched as a programmatic
+ * dependent of the discovery, so its prologue overlaps discovery's tail, and
+ * it takes its work units (request, KV group, query block, M-tile pair) from
+ * a device queue in the workspace, longest query blocks first, instead of a
+ * static stride. workspace: fp_workspace_size(p) bytes as for fp_discover.
+ * Outputs are identical to the three separate calls.
+ */
+fp_status_t fp_prefill(const fp_params_t* p, const void* q, const void* k, const void* v, uint32_t* mask,
+                       int32_t* idx, int32_t* cnt, void* o, float* lse, void* workspace, size_t ws_bytes,
+                       void* stream);
+
+/*
  * Discovery and compaction without a caller-provided workspace: the same
  * kernels and outputs as fp_discover_compact, with the pooled-Q/K scratch
  * taken from a fixed device array inside the library. The paper has no

@@ -426,3 +426,44 @@ def test_per_head_with_every_head_selecting_equals_group_mode():
     d2.attend()
     assert torch.equal(d1.bufs.cnt, d2.bufs.cnt)
     assert torch.equal(d1.bufs.o, d2.bufs.o) and torch.equal(d1.bufs.lse, d2.bufs.lse)
+
+
+# ----------------------------------------------------------------------------- single-call path
+def _prefill_case(case):
+    if case == "contig":
+        w = _case("qwen30b_128k", 4000)
+        return w, _inputs(w), False
+    if case == "fp8":
+        w = _case("qwen30b_128k", 3000)
+        return w, _inputs(w, True), False
+    if case == "paged":
+        w = W["paged_varlen"].with_(seqlens=(900, 2100, 64))
+        return w, _inputs(w), False
+    if case == "chunked":
+        w = W["paged_varlen"]
+        return w, wl.make_chunked_inputs(w, (1500, 700), (600, 700)), False
+    w = _case("tiny2k")
+    return w, _inputs(w), True
+
+
+@pytest.mark.parametrize("case", ["contig", "fp8", "paged", "chunked", "per_head"])
+def test_prefill_single_call_equals_separate_calls(case):
+    """fp_prefill (device work queue, dependent launch) gives exactly the outputs
+    of fp_discover_compact followed by the attention call."""
+    from block_sparse_long_blocks_b200 import binding as fb
+    w, inp, per_head = _prefill_case(case)
+    a = H.Device(w, inp, per_head=per_head)
+    a.discover()
+    a.attend()
+    b = H.Device(w, inp, per_head=per_head)
+    b.bufs.o.zero_()
+    b.bufs.lse.fill_(float("nan"))
+    fb.fp_prefill(b.p, b.q, b.k, b.v, b.bufs.mask, b.bufs.idx, b.bufs.cnt, b.bufs.o, b.bufs.workspace, b.bufs.lse)
+    torch.cuda.synchronize()
+    assert b.status() == 0
+    assert torch.equal(a.bufs.cnt, b.bufs.cnt) and torch.equal(a.bufs.mask, b.bufs.mask)
+    assert a.lists() == b.lists()
+    if per_head:
+        assert torch.equal(a.head_bits, b.head_bits)
+    assert torch.equal(a.bufs.o, b.bufs.o)
+    assert torch.equal(torch.nan_to_num(a.bufs.lse, nan=7.0), torch.nan_to_num(b.bufs.lse, nan=7.0))
