@@ -97,7 +97,6 @@ Geometry geometry(const fp_params_t* p) {
   g.B = p->block;
   g.Nmax = ceil_div(g.L, g.B);
   g.Wmax = ceil_div(g.Nmax, 32);
-  g.Npad = (g.Nmax + 3) / 4 * 4;
   g.Sb = ceil_div(p->sink_tokens, g.B);
   g.Wb = ceil_div(p->window_tokens, g.B);
   if (g.Wb < 1) g.Wb = 1;
@@ -122,12 +121,14 @@ Geometry geometry(const fp_params_t* p) {
   return g;
 }
 
-size_t qbar_floats(const Geometry& g) { return (size_t)g.R * g.Nmax * g.Hq * 128; }
-size_t kbar_floats(const Geometry& g) { return (size_t)g.R * g.Hkv * 128 * g.Npad; }
+// Workspace: pooled query planes, pooled key planes (256-byte aligned), then
+// the attention work-queue counter.
+size_t pad256(size_t bytes) { return (bytes + 255) / 256 * 256; }
+size_t pooled_q_bytes(const Geometry& g) { return pad256(3 * pooled_q_elems(g) * sizeof(__nv_bfloat16)); }
+size_t pooled_k_bytes(const Geometry& g) { return pad256(3 * pooled_k_elems(g) * sizeof(__nv_bfloat16)); }
 
-// The attention work-queue counter lives right after the pooled tensors.
 int* queue_slot(const Geometry& g, void* ws) {
-  return reinterpret_cast<int*>(static_cast<float*>(ws) + (qbar_floats(g) + 63) / 64 * 64 + kbar_floats(g));
+  return reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + pooled_q_bytes(g) + pooled_k_bytes(g));
 }
 
 fp_status_t discover_impl(const fp_params_t* p, const void* q, const void* k, uint32_t* mask, int32_t* idx,
@@ -141,18 +142,15 @@ fp_status_t discover_impl(const fp_params_t* p, const void* q, const void* k, ui
     return FP_ERR_ALIGNMENT;
   if (!ws || !aligned(ws, 256) || ws_bytes < fp_workspace_size(p)) return FP_ERR_WORKSPACE;
   Geometry g = geometry(p);
-  if (score_smem_bytes(g) > 227 * 1024) return FP_ERR_UNSUPPORTED;
   g.status = status_ptr();
   if (!g.status) return cuda_fail("device status symbol", cudaGetLastError());
   if (zero_queue) g.attn_queue = queue_slot(g, ws);
-  float* qbar = static_cast<float*>(ws);
-  float* kbarT = qbar + (qbar_floats(g) + 63) / 64 * 64;
+  __nv_bfloat16* qpl = static_cast<__nv_bfloat16*>(ws);
+  __nv_bfloat16* kpl = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + pooled_q_bytes(g));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_pool(g, q, k, qbar, kbarT, s);
+  const cudaError_t e = launch_pool(g, q, k, qpl, kpl, s);
   if (e != cudaSuccess) return cuda_fail("pool launch", e);
-  e = launch_score(g, qbar, kbarT, mask, idx, cnt, s);
-  if (e != cudaSuccess) return cuda_fail("score launch", e);
-  return FP_OK;
+  return launch_score(g, qpl, kpl, mask, idx, cnt, s);
 }
 
 fp_status_t attention_impl(const fp_params_t* p, bool paged, const void* q, const void* k, const void* v,
@@ -180,7 +178,7 @@ extern "C" {
 size_t fp_workspace_size(const fp_params_t* p) {
   if (validate(p, false) != FP_OK) return 0;
   const Geometry g = geometry(p);
-  return ((qbar_floats(g) + 63) / 64 * 64 + kbar_floats(g)) * sizeof(float) + 256;  // + work-queue counter
+  return pooled_q_bytes(g) + pooled_k_bytes(g) + 256;  // + work-queue counter
 }
 
 size_t fp_mask_words(const fp_params_t* p) {

@@ -31,7 +31,6 @@
 
 #include <climits>
 #include <cstdio>
-#include <mutex>
 
 #include "internal.cuh"
 #include "sm100.cuh"
@@ -77,7 +76,11 @@ template <bool FP8>
 struct MaxOffset {
   static constexpr float value = FP8 ? (float)FP_E4M3_MAX_OFFSET : 0.0f;
 };
-constexpr int kSmemBudget = 200 * 1024;
+// Shared memory for the Q tiles and the K/V rings (the opt-in maximum per CTA is 227 KB).
+#ifndef FP_SMEM_BUDGET_KB
+#define FP_SMEM_BUDGET_KB 200
+#endif
+constexpr int kSmemBudget = FP_SMEM_BUDGET_KB * 1024;
 
 // 2^x with the MUFU.EX2 instruction (flush-to-zero, ~2 ulp); 2^-inf = +0.
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -214,18 +217,24 @@ struct Cfg {
   static constexpr int Q_TILE = DCH * 128 * 128;          // bytes per 128-row M-tile
   static constexpr int KV_CHUNK = BLK * 128;              // bytes per d-chunk of a K/V tile
   static constexpr int KV_TILE = DCH * KV_CHUNK;
-  static constexpr int STAGES_RAW = (kSmemBudget - 2 * Q_TILE) / (2 * KV_TILE);
-  static constexpr int STAGES = STAGES_RAW > 4 ? 4 : STAGES_RAW;
+  // K/V ring slots within the budget; an odd slot goes to K, whose tile is
+  // consumed about one visit before the V tile of the same block
+  static constexpr int TILES_RAW = (kSmemBudget - 2 * Q_TILE) / KV_TILE;
+  static constexpr int TILES = TILES_RAW > 8 ? 8 : TILES_RAW;
+  static constexpr int V_STAGES = TILES / 2;
+  static constexpr int K_STAGES = TILES - V_STAGES;
   static constexpr int KSTEP_BYTES = 32;                  // K extent of one MMA (16 bf16 / 32 e4m3)
   static constexpr int QK_STEPS = 128 * ES / KSTEP_BYTES; // 8 (bf16) / 4 (e4m3)
   static constexpr int PV_KEYS = KSTEP_BYTES / ES;        // keys per PV MMA: 16 / 32
   static constexpr int PV_STEPS = BLK / PV_KEYS;
-  static constexpr int NUM_BARS = 2 + 4 * STAGES + 6 + 1 + 2 * kUnitRing;
-  static constexpr int SMEM_USED = 1024 + 2 * Q_TILE + 2 * STAGES * KV_TILE + NUM_BARS * 8 + 16 + 4 * kUnitRing;
+  static constexpr int NUM_BARS = 2 + 2 * (K_STAGES + V_STAGES) + 6 + 1 + 2 * kUnitRing;
+  static constexpr int SMEM_USED =
+      1024 + 2 * Q_TILE + (K_STAGES + V_STAGES) * KV_TILE + NUM_BARS * 8 + 16 + 4 * kUnitRing;
   // more than half of the SM's shared memory: one CTA per SM, so the CTA's
   // 512-column TMEM allocation never waits for a co-resident CTA
   static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
-  static_assert(STAGES >= 2, "shared memory budget too small");
+  static_assert(V_STAGES >= 2, "shared memory budget too small");
+  static_assert(SMEM <= 227 * 1024, "beyond the per-CTA shared memory limit");
 };
 
 // Work units reach the roles either by a static stride over the persistent
@@ -349,20 +358,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     sparse_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   using C = Cfg<FP8, BLK>;
-  constexpr int S = C::STAGES;
+  constexpr int KS = C::K_STAGES, VS = C::V_STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + 2 * C::Q_TILE;
-  uint8_t* sV = sK + S * C::KV_TILE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + S * C::KV_TILE);
+  uint8_t* sV = sK + KS * C::KV_TILE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VS * C::KV_TILE);
   uint64_t* q_full = bars;
   uint64_t* q_empty = bars + 1;
   uint64_t* k_full = bars + 2;
-  uint64_t* k_empty = k_full + S;
-  uint64_t* v_full = k_empty + S;
-  uint64_t* v_empty = v_full + S;
-  uint64_t* s_full = v_empty + S;  // [2]
+  uint64_t* k_empty = k_full + KS;
+  uint64_t* v_full = k_empty + KS;
+  uint64_t* v_empty = v_full + VS;
+  uint64_t* s_full = v_empty + VS;  // [2]
   uint64_t* p_full = s_full + 2;   // [2]
   uint64_t* o_full = p_full + 2;   // [2]
   uint64_t* drain = o_full + 2;
@@ -378,9 +387,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int s = 0; s < S; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(k_full + s, 1);
       mbar_init(k_empty + s, 1);
+    }
+    for (int s = 0; s < VS; ++s) {
       mbar_init(v_full + s, 1);
       mbar_init(v_empty + s, 1);
     }
@@ -446,14 +457,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++qn;
         for (int n = 0; n < U.count && ok; ++n) {
           const int j = list_entry(a, U, n);
-          int st = (int)(kt % S);
-          ok = mbar_wait(k_empty + st, (uint32_t)((kt / S) & 1) ^ 1u, abort_flag, g.status, FP_DEV_TIMEOUT);
+          int st = (int)(kt % KS);
+          ok = mbar_wait(k_empty + st, (uint32_t)((kt / KS) & 1) ^ 1u, abort_flag, g.status, FP_DEV_TIMEOUT);
           if (!ok) break;
           mbar_arrive_expect_tx(k_full + st, C::KV_TILE);
           load_kv_tile<FP8, BLK, PAGED>(sK + st * C::KV_TILE, &tmK, k_full + st, a, U, j);
           ++kt;
-          st = (int)(vt % S);
-          ok = mbar_wait(v_empty + st, (uint32_t)((vt / S) & 1) ^ 1u, abort_flag, g.status, FP_DEV_TIMEOUT);
+          st = (int)(vt % VS);
+          ok = mbar_wait(v_empty + st, (uint32_t)((vt / VS) & 1) ^ 1u, abort_flag, g.status, FP_DEV_TIMEOUT);
           if (!ok) break;
           mbar_arrive_expect_tx(v_full + st, C::KV_TILE);
           load_kv_tile<FP8, BLK, PAGED>(sV + st * C::KV_TILE, &tmV, v_full + st, a, U, j);
@@ -463,10 +474,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (*abort_flag) {
         // let every copy this CTA issued land before the shared memory is released
         int never = 0;
-        for (long long t = kt - 1; t >= 0 && t >= kt - S; --t)
-          mbar_wait(k_full + (int)(t % S), (uint32_t)((t / S) & 1), (volatile int*)&never, g.status, 0u);
-        for (long long t = vt - 1; t >= 0 && t >= vt - S; --t)
-          mbar_wait(v_full + (int)(t % S), (uint32_t)((t / S) & 1), (volatile int*)&never, g.status, 0u);
+        for (long long t = kt - 1; t >= 0 && t >= kt - KS; --t)
+          mbar_wait(k_full + (int)(t % KS), (uint32_t)((t / KS) & 1), (volatile int*)&never, g.status, 0u);
+        for (long long t = vt - 1; t >= 0 && t >= vt - VS; --t)
+          mbar_wait(v_full + (int)(t % VS), (uint32_t)((t / VS) & 1), (volatile int*)&never, g.status, 0u);
         if (qn > 0) mbar_wait(q_full, (uint32_t)((qn - 1) & 1), (volatile int*)&never, g.status, 0u);
       }
     }
@@ -516,8 +527,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = mbar_wait(q_full, (uint32_t)(qn & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
         if (!ok) break;
         ++qn;
-        int kst = (int)(kt % S);
-        ok = mbar_wait(k_full + kst, (uint32_t)((kt / S) & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
+        int kst = (int)(kt % KS);
+        ok = mbar_wait(k_full + kst, (uint32_t)((kt / KS) & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
         if (!ok) break;
         tc_fence_after();
         issue_qk(0, kst);
@@ -528,8 +539,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++kt;
         if (U.count == 1) umma_commit(q_empty);
         for (int n = 0; n < U.count; ++n) {
-          const int vst = (int)(vt % S);
-          ok = mbar_wait(v_full + vst, (uint32_t)((vt / S) & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
+          const int vst = (int)(vt % VS);
+          ok = mbar_wait(v_full + vst, (uint32_t)((vt / VS) & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
           if (!ok) break;
           ok = mbar_wait(p_full + 0, (uint32_t)(pn[0] & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
           if (!ok) break;
@@ -538,8 +549,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           issue_pv(0, vst, n > 0);
           const bool more = n + 1 < U.count;
           if (more) {
-            kst = (int)(kt % S);
-            ok = mbar_wait(k_full + kst, (uint32_t)((kt / S) & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
+            kst = (int)(kt % KS);
+            ok = mbar_wait(k_full + kst, (uint32_t)((kt / KS) & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
             if (!ok) break;
             tc_fence_after();
             issue_qk(0, kst);
@@ -773,43 +784,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
 bool encode(CUtensorMap* m, bool fp8, int rank, const void* base, const cuuint64_t* dims, const cuuint64_t* strides,
             const cuuint32_t* box) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) {
-    set_last_error("cuTensorMapEncodeTiled lookup", 0, "driver entry point not found");
-    return false;
-  }
-  cuuint32_t es[4] = {1, 1, 1, 1};
-  const CUresult r = fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
-                        const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) {
-    char buf[160];
-    snprintf(buf, sizeof(buf), "rank %d dims %llu,%llu,%llu box %u,%u,%u", rank, (unsigned long long)dims[0],
-             (unsigned long long)dims[1], (unsigned long long)dims[2], box[0], box[1], box[2]);
-    set_last_error("cuTensorMapEncodeTiled", (int)r, buf);
-    return false;
-  }
-  return true;
+  return encode_tiled(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, dims,
+                      strides, box);
 }
 
 int sm_count() {

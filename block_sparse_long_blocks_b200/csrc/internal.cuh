@@ -1,6 +1,8 @@
 // Internal (non-ABI) definitions shared by the library's translation units.
 #pragma once
 
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -16,7 +18,6 @@ struct Geometry {
   int B;          // block size (tokens)
   int Nmax;       // ceil(L / B)
   int Wmax;       // ceil(Nmax / 32) mask words per row
-  int Npad;       // Nmax rounded up to a multiple of 4 (stride of the transposed pooled K)
   int Sb, Wb;     // sink / window in blocks
   float scale;    // softmax scale
   float thr;      // ln(alpha) (-inf for alpha == 0)
@@ -80,10 +81,16 @@ __host__ __device__ __forceinline__ long long row_index(int r, int kvh, int i, i
   return ((long long)r * Hkv + kvh) * Nmax + i;
 }
 
-// host launchers (each returns a cudaError_t of its launch)
-cudaError_t launch_pool(const Geometry& g, const void* q, const void* k, float* qbar, float* kbarT,
+// Pooled tensors in the workspace, each as three bf16 planes (hi, mid, lo):
+// queries [3][R * Nmax][Hq][128], keys [3][R * Hkv][Nmax][128]. Elements per plane:
+size_t pooled_q_elems(const Geometry& g);
+size_t pooled_k_elems(const Geometry& g);
+
+// host launchers
+cudaError_t launch_pool(const Geometry& g, const void* q, const void* k, __nv_bfloat16* qpl, __nv_bfloat16* kpl,
                         cudaStream_t s);
-cudaError_t launch_score(const Geometry& g, const float* qbar, const float* kbarT, uint32_t* mask,
+// Returns FP_OK, FP_ERR_UNSUPPORTED or FP_ERR_CUDA (with the failing step recorded).
+fp_status_t launch_score(const Geometry& g, const __nv_bfloat16* qpl, const __nv_bfloat16* kpl, uint32_t* mask,
                          int32_t* idx, int32_t* cnt, cudaStream_t s);
 cudaError_t launch_compact(const Geometry& g, const uint32_t* mask, int32_t* idx, int32_t* cnt,
                            cudaStream_t s);
@@ -94,7 +101,11 @@ fp_status_t launch_attention(const Geometry& g, const void* q, const void* k, co
                              const int32_t* idx, const int32_t* cnt, void* o, float* lse,
                              cudaStream_t s, int* queue, bool pdl);
 
-size_t score_smem_bytes(const Geometry& g);
+// cuTensorMapEncodeTiled (through the runtime's driver entry point) with
+// 128-byte swizzle, 256-byte L2 promotion and zero fill outside the tensor.
+// On failure records the step (fp_last_error) and returns false.
+bool encode_tiled(CUtensorMap* map, CUtensorMapDataType type, int rank, const void* base, const cuuint64_t* dims,
+                  const cuuint64_t* strides, const cuuint32_t* box);
 
 // Records the failing step of the calling thread's last FP_ERR_CUDA (read by fp_last_error).
 void set_last_error(const char* step, int code, const char* detail);

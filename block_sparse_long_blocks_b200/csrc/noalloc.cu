@@ -19,8 +19,8 @@
 namespace fp {
 namespace {
 
-// 32 MiB: the pooled Q and K (float32) of one 128K-token sequence with 32
-// query and 4 KV heads at block 128 need 18.9 MB.
+// 32 MiB: the pooled Q and K (three bf16 planes each) of one 128K-token
+// sequence with 32 query and 4 KV heads at block 128 need 28.3 MB.
 constexpr size_t kStaticScratchBytes = 32ull << 20;
 constexpr int kMaxScratchDevices = 64;
 

@@ -64,8 +64,10 @@
  *   cnt[(r * Hkv + g) * Nmax + i] strictly ascending block indices (capacity
  *   i + 1). Rows i >= N_r have cnt = 0.
  * - Thresholding happens in float32: keep iff s - rowmax >= ln(alpha), with
- *   s = softmax_scale * (pooled q . pooled k). Blocks whose exact probability
- *   lies within ~1e-5 relative of alpha may be decided either way.
+ *   s = softmax_scale * (pooled q . pooled k); the dot products are formed on
+ *   the tensor cores from three-part bf16 splits of the float32 means, to
+ *   float32 accuracy. Blocks whose exact probability lies within ~1e-5
+ *   relative of alpha may be decided either way.
  */
 #ifndef FLASHPREFILL_H_
 #define FLASHPREFILL_H_
@@ -119,7 +121,9 @@ typedef struct {
   uint8_t* head_bits;         /* per-head selection: device uint8 [fp_list_capacity(p)] or NULL (see below) */
 } fp_params_t;
 
-/* Bytes of device scratch fp_discover needs (pooled Q and K, float32). */
+/* Bytes of device scratch fp_discover needs: the pooled Q and K, each pooled
+ * float32 value stored as three bf16 parts (hi + mid + lo), plus 256 bytes
+ * for fp_prefill's work-queue counter. */
 size_t fp_workspace_size(const fp_params_t* p);
 /* Number of uint32 words of the block mask: R * Hkv * Nmax * ceil(Nmax / 32). */
 size_t fp_mask_words(const fp_params_t* p);

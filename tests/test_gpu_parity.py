@@ -66,6 +66,29 @@ def test_discovery_matches_oracle(name, L, alpha, fused):
     _mask_matches_lists(dev)
 
 
+# Cases spanning several 128-block column tiles of the scoring kernel (ragged
+# last tile) and the group sizes it specialises.
+TILE_CASES = [
+    ("qwen30b_128k", 40000, {}),                     # G=8, Nmax=313: three column tiles
+    ("tiny2k", 10000, {}),                           # B=64, G=4, Nmax=157
+    ("qwen7b_32k", 20000, {}),                       # G=7: 18 query blocks x 7 heads per tile
+    ("qwen30b_128k", 9000, {"hkv": 2}),              # G=16
+    ("qwen30b_128k", 9000, {"hq": 4}),               # G=1: 128 query blocks per tile
+    ("qwen30b_128k", 20000, {"hq": 6, "hkv": 2}),    # G=3
+]
+
+
+@pytest.mark.parametrize("name,L,kw", TILE_CASES)
+def test_discovery_column_tiles_and_groups(name, L, kw):
+    w = _case(name, L, **kw)
+    inp = _inputs(w)
+    dev = H.Device(w, inp)
+    dev.discover()
+    assert dev.status() == 0
+    H.compare_lists(H.oracle_discovery(w, inp), dev.lists())
+    _mask_matches_lists(dev)
+
+
 @pytest.mark.parametrize("name,L", [("tiny2k", None), ("qwen30b_128k", 4096)])
 def test_discovery_fp8_matches_oracle(name, L):
     w = _case(name, L)
@@ -411,6 +434,40 @@ def test_per_head_selection_matches_oracle(name, L, fp8):
     else:
         assert e.max() <= H.BF16_MAX and e.mean() <= H.BF16_MEAN
     assert np.abs(gl_ - lse).max() <= (2e-3 if fp8 else 5e-3)
+
+
+def _check_head_bits(dev, w, orc):
+    """Device head bits equal the oracle's per-head keep bits on every list entry
+    the two lists share exactly (borderline rows are left to compare_lists)."""
+    Sb, Wb = oracle.forced_blocks(w.sink_tokens, w.window_tokens, w.block)
+    keep = [oracle.head_masks(o["qbar"], o["kbar"], o["scale"], w.alpha, Sb, Wb) for o in orc]
+    want = H.head_bits_array(dev.cfg, [o["lists"] for o in orc], keep, w.group)
+    got = dev.head_bits.cpu().numpy()
+    gl = dev.lists()
+    N = dev.cfg.nmax
+    tri = N * (N + 1) // 2
+    for g in range(w.hkv):
+        for i in range(N):
+            if gl[0][g][i] != [int(x) for x in orc[0]["lists"][g][i]]:
+                continue
+            base = g * tri + i * (i + 1) // 2
+            n = len(gl[0][g][i])
+            if not np.array_equal(got[base:base + n], want[base:base + n]):
+                b = oracle.row_borderline(orc[0]["qbar"], orc[0]["kbar"], orc[0]["scale"], w.alpha, g, i,
+                                          H.BORDER_REL)
+                bad = [gl[0][g][i][k] for k in range(n) if got[base + k] != want[base + k]]
+                assert set(bad) <= b, (g, i, bad)
+
+
+def test_per_head_bits_span_column_tiles():
+    w = _case("qwen30b_128k", 40000)
+    inp = _inputs(w)
+    dev = H.Device(w, inp, per_head=True)
+    dev.discover()
+    assert dev.status() == 0
+    orc = H.oracle_discovery(w, inp)
+    H.compare_lists(orc, dev.lists())
+    _check_head_bits(dev, w, orc)
 
 
 def test_per_head_with_every_head_selecting_equals_group_mode():
