@@ -46,11 +46,13 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 // Launched at 168 registers/thread (384 x 168 = 64512). The softmax warpgroups
 // then raise their limit and the producer/MMA warpgroup lowers its own:
-// 2 x 128 x 200 + 128 x 96 = 63488 <= 64512, and per SM sub-partition (three
-// warps each) 2 x 32 x 200 + 32 x 96 = 15872 <= 16384.
+// 2 x 128 x 200 + 128 x 104 = 64512 <= 64512, and per SM sub-partition (three
+// warps each) 2 x 32 x 200 + 32 x 104 = 16128 <= 16384. (At 96 the MMA
+// issuer's loop spills.)
 constexpr uint32_t kSoftmaxRegs = 200;
-constexpr uint32_t kControlRegs = 96;
+constexpr uint32_t kControlRegs = 104;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * 168, "register split exceeds the launch");
+static_assert(2 * 32 * kSoftmaxRegs + 32 * kControlRegs <= 16384, "register split exceeds an SM sub-partition");
 // The reference max is raised only when a tile's max exceeds it by more than
 // this (log2 units); P is then at most 2^threshold. e4m3 P must stay below 448.
 // bf16 P, the float32 row sum and the float32 TMEM accumulators have float32's
@@ -492,13 +494,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       long long pn[2] = {0, 0};
       bool ok = true;
 
+      // Descriptors of the tiles' first bytes; an operand at byte offset `off`
+      // within the CTA's shared window is base + off / 16 (the start-address
+      // field cannot carry: every address is below 256 KB).
+      const uint64_t dQ = smem_desc_sw128(sQa, 16, 1024);
+      const uint64_t dK = smem_desc_sw128(sKa, 16, 1024);
+      const uint64_t dV = smem_desc_sw128(sVa, C::KV_CHUNK, 1024);
       auto issue_qk = [&](int mt, int kst) {
+        const uint64_t a0 = dQ + (uint64_t)((mt * C::Q_TILE) >> 4);
+        const uint64_t b0 = dK + (uint64_t)((kst * C::KV_TILE) >> 4);
 #pragma unroll
         for (int ks = 0; ks < C::QK_STEPS; ++ks) {
           const uint32_t boff = (uint32_t)(ks * C::KSTEP_BYTES);
           const uint32_t ch = boff / 128, in = boff % 128;
-          const uint64_t ad = smem_desc_sw128(sQa + mt * C::Q_TILE + ch * 128 * 128 + in, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sKa + kst * C::KV_TILE + ch * C::KV_CHUNK + in, 16, 1024);
+          const uint64_t ad = a0 + ((ch * 128 * 128 + in) >> 4);
+          const uint64_t bd = b0 + ((ch * C::KV_CHUNK + in) >> 4);
           if (FP8) umma_f8_ss(tmem + mt * 128, ad, bd, idesc_qk, ks > 0);
           else umma_f16_ss(tmem + mt * 128, ad, bd, idesc_qk, ks > 0);
         }
@@ -506,13 +516,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P occupies the first columns of the M-tile's S region: bf16 pairs, or for
       // e4m3 a high plane (BLK/4 columns) followed by the residual plane.
       auto issue_pv = [&](int mt, int vst, bool acc) {
+        const uint64_t b0 = dV + (uint64_t)((vst * C::KV_TILE) >> 4);
 #pragma unroll
         for (int plane = 0; plane < (FP8 ? 2 : 1); ++plane) {
 #pragma unroll
           for (int ks = 0; ks < C::PV_STEPS; ++ks) {
             const uint32_t a_t = tmem + mt * 128 + plane * (BLK / 4) + ks * (C::PV_KEYS * C::ES / 4);
-            const uint64_t bd =
-                smem_desc_sw128(sVa + vst * C::KV_TILE + ks * C::PV_KEYS * 128, C::KV_CHUNK, 1024);
+            const uint64_t bd = b0 + ((ks * C::PV_KEYS * 128) >> 4);
             const uint32_t accum = (acc || ks > 0 || plane > 0) ? 1u : 0u;
             if (FP8) umma_f8_ts(tmem + 256 + mt * 128, a_t, bd, idesc_pv, accum);
             else umma_f16_ts(tmem + 256 + mt * 128, a_t, bd, idesc_pv, accum);
@@ -700,17 +710,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           // P = hi + lo, both e4m3: the residual plane keeps the weights' relative
           // error near 2^-8 instead of e4m3's 2^-4. Planes: hi in columns
-          // [0, BLK/4), lo in [BLK/4, BLK/2); packed 64 values (16 columns) at a time.
+          // [0, BLK/4), lo in [BLK/4, BLK/2); packed 32 values (8 columns) at a time.
 #pragma unroll
-          for (int c = 0; c < BLK / 64; ++c) {
-            uint32_t phi[16], plo[16];
+          for (int c = 0; c < BLK / 32; ++c) {
+            uint32_t phi[8], plo[8];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
+            for (int e = 0; e < 8; ++e) {
               uint32_t h32 = 0, l32 = 0;
 #pragma unroll
               for (int q = 0; q < 2; ++q) {
                 float x0, x1;
-                exp2_pair(s[64 * c + 4 * e + 2 * q], s[64 * c + 4 * e + 2 * q + 1], sl2, m_ref, sl2x2, negm2,
+                exp2_pair(s[32 * c + 4 * e + 2 * q], s[32 * c + 4 * e + 2 * q + 1], sl2, m_ref, sl2x2, negm2,
                           emulated_pair(2 * e + q), x0, x1);
                 uint32_t h, r;
                 e4m3_split2(x0, x1, h, r);
@@ -727,8 +737,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               phi[e] = h32;
               plo[e] = l32;
             }
-            tmem_st16(tS + 16 * c, phi);
-            tmem_st16(tS + BLK / 4 + 16 * c, plo);
+            tmem_st8(tS + 8 * c, phi);
+            tmem_st8(tS + BLK / 4 + 8 * c, plo);
           }
         }
         l += (lsum0 + lsum1) + (lsum2 + lsum3);
