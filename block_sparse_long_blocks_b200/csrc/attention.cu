@@ -229,7 +229,7 @@ struct Cfg {
   static constexpr int QK_STEPS = 128 * ES / KSTEP_BYTES; // 8 (bf16) / 4 (e4m3)
   static constexpr int PV_KEYS = KSTEP_BYTES / ES;        // keys per PV MMA: 16 / 32
   static constexpr int PV_STEPS = BLK / PV_KEYS;
-  static constexpr int NUM_BARS = 2 + 2 * (K_STAGES + V_STAGES) + 6 + 1 + 2 * kUnitRing;
+  static constexpr int NUM_BARS = 2 + 2 * (K_STAGES + V_STAGES) + 8 + 1 + 2 * kUnitRing;
   static constexpr int SMEM_USED =
       1024 + 2 * Q_TILE + (K_STAGES + V_STAGES) * KV_TILE + NUM_BARS * 8 + 16 + 4 * kUnitRing;
   // more than half of the SM's shared memory: one CTA per SM, so the CTA's
@@ -374,8 +374,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_full = k_empty + KS;
   uint64_t* v_empty = v_full + VS;
   uint64_t* s_full = v_empty + VS;  // [2]
-  uint64_t* p_full = s_full + 2;   // [2]
-  uint64_t* o_full = p_full + 2;   // [2]
+  uint64_t* p_full = s_full + 2;   // [M-tile][half of the keys]
+  uint64_t* o_full = p_full + 4;   // [2]
   uint64_t* drain = o_full + 2;
   uint64_t* unit_full = drain + 1;             // [kUnitRing]
   uint64_t* unit_empty = unit_full + kUnitRing;  // [kUnitRing]
@@ -399,7 +399,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int m = 0; m < 2; ++m) {
       mbar_init(s_full + m, 1);
-      mbar_init(p_full + m, 128);
+      mbar_init(p_full + 2 * m, 128);
+      mbar_init(p_full + 2 * m + 1, 128);
       mbar_init(o_full + m, 1);
     }
     mbar_init(drain, 1);
@@ -515,12 +516,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // P occupies the first columns of the M-tile's S region: bf16 pairs, or for
       // e4m3 a high plane (BLK/4 columns) followed by the residual plane.
-      auto issue_pv = [&](int mt, int vst, bool acc) {
+      auto issue_pv = [&](int mt, int vst, bool acc, int hf) {
         const uint64_t b0 = dV + (uint64_t)((vst * C::KV_TILE) >> 4);
 #pragma unroll
         for (int plane = 0; plane < (FP8 ? 2 : 1); ++plane) {
 #pragma unroll
-          for (int ks = 0; ks < C::PV_STEPS; ++ks) {
+          for (int ks = hf * (C::PV_STEPS / 2); ks < (hf + 1) * (C::PV_STEPS / 2); ++ks) {
             const uint32_t a_t = tmem + mt * 128 + plane * (BLK / 4) + ks * (C::PV_KEYS * C::ES / 4);
             const uint64_t bd = b0 + ((ks * C::PV_KEYS * 128) >> 4);
             const uint32_t accum = (acc || ks > 0 || plane > 0) ? 1u : 0u;
@@ -554,25 +555,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           ok = mbar_wait(p_full + 0, (uint32_t)(pn[0] & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
           if (!ok) break;
-          ++pn[0];
           tc_fence_after();
-          issue_pv(0, vst, n > 0);
+          issue_pv(0, vst, n > 0, 0);
+          // the next K tile is waited for while softmax 0 finishes its second half,
+          // so S0(n+1) follows PV0(n) without a gap
           const bool more = n + 1 < U.count;
           if (more) {
             kst = (int)(kt % KS);
             ok = mbar_wait(k_full + kst, (uint32_t)((kt / KS) & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
             if (!ok) break;
-            tc_fence_after();
+          }
+          ok = mbar_wait(p_full + 1, (uint32_t)(pn[0] & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
+          if (!ok) break;
+          ++pn[0];
+          tc_fence_after();
+          issue_pv(0, vst, true, 1);
+          if (more) {
             issue_qk(0, kst);
             umma_commit(s_full + 0);
           } else {
             umma_commit(o_full + 0);
           }
-          ok = mbar_wait(p_full + 1, (uint32_t)(pn[1] & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
+          ok = mbar_wait(p_full + 2, (uint32_t)(pn[1] & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(1, vst, n > 0, 0);
+          ok = mbar_wait(p_full + 3, (uint32_t)(pn[1] & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
           if (!ok) break;
           ++pn[1];
           tc_fence_after();
-          issue_pv(1, vst, n > 0);
+          issue_pv(1, vst, true, 1);
           umma_commit(v_empty + vst);
           ++vt;
           if (more) {
@@ -631,36 +643,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         ++sn;
         tc_fence_after();
+        // S in two halves: the second half's TMEM load is in flight while the
+        // first half is masked and reduced
         float s[BLK];
+        const bool diag = last_is_diag && n == U.count - 1;  // keys after the query are masked
+        const bool hmask = !((hb >> hh) & 1u);               // block not kept by this row's head
+        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
         {
           uint32_t sr[BLK];
 #pragma unroll
-          for (int c = 0; c < BLK / 32; ++c) tmem_ld32(tS + c * 32, sr + c * 32);
+          for (int c = 0; c < BLK / 64; ++c) tmem_ld32(tS + c * 32, sr + c * 32);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < BLK; ++c) s[c] = __uint_as_float(sr[c]);
-        }
-        if (last_is_diag && n == U.count - 1) {  // diagonal block: keys after the query are masked
+          for (int c = BLK / 64; c < BLK / 32; ++c) tmem_ld32(tS + c * 32, sr + c * 32);
 #pragma unroll
-          for (int c = 0; c < BLK; ++c)
-            if (c > qtok) s[c] = -INFINITY;
-        }
-        if (!((hb >> hh) & 1u)) {
+          for (int hf = 0; hf < 2; ++hf) {
+            if (hf == 1) tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < BLK; ++c) s[c] = -INFINITY;
-        }
-        float mx;
-        {
-          float m0 = fmaxf(s[0], s[1]), m1 = fmaxf(s[2], s[3]), m2 = fmaxf(s[4], s[5]), m3 = fmaxf(s[6], s[7]);
+            for (int c = hf * (BLK / 2); c < (hf + 1) * (BLK / 2); ++c) s[c] = __uint_as_float(sr[c]);
+            if (diag || hmask) {
 #pragma unroll
-          for (int c = 8; c < BLK; c += 8) {
-            m0 = fmax3(m0, s[c], s[c + 1]);
-            m1 = fmax3(m1, s[c + 2], s[c + 3]);
-            m2 = fmax3(m2, s[c + 4], s[c + 5]);
-            m3 = fmax3(m3, s[c + 6], s[c + 7]);
+              for (int c = hf * (BLK / 2); c < (hf + 1) * (BLK / 2); ++c)
+                if (hmask || c > qtok) s[c] = -INFINITY;
+            }
+#pragma unroll
+            for (int c = hf * (BLK / 2); c < (hf + 1) * (BLK / 2); c += 8) {
+              m0 = fmax3(m0, s[c], s[c + 1]);
+              m1 = fmax3(m1, s[c + 2], s[c + 3]);
+              m2 = fmax3(m2, s[c + 4], s[c + 5]);
+              m3 = fmax3(m3, s[c + 6], s[c + 7]);
+            }
           }
-          mx = fmax3(m0, m1, fmaxf(m2, m3));
         }
+        const float mx = fmax3(m0, m1, fmaxf(m2, m3));
         const float m_new = fmaxf(m_ref, mx * sl2);
         const bool need = m_new > m_ref + RescaleThreshold<FP8>::value;
         const float f = need ? fast_exp2(m_ref - (m_new - MaxOffset<FP8>::value)) : 1.f;
@@ -690,22 +705,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         // (m_ref stays -inf while every visited block so far was masked for this row)
         const float negm = m_ref == -INFINITY ? 0.f : -m_ref;
         const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(negm, negm);
+        // P goes out in two halves of the visited block's keys; the MMA issuer
+        // starts O += P V on the first half while the second is computed.
         if constexpr (!FP8) {
+          constexpr int HALF = BLK / 2;              // keys per half
+          constexpr int CH = HALF < 64 ? HALF : 64;  // keys per TMEM store
 #pragma unroll
-          for (int c = 0; c < BLK / 64; ++c) {
-            uint32_t pk[32];
+          for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              float p0, p1;
-              exp2_pair(s[c * 64 + 2 * e], s[c * 64 + 2 * e + 1], sl2, m_ref, sl2x2, negm2, emulated_pair(e), p0,
-                        p1);
-              const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-              const uint32_t u = *reinterpret_cast<const uint32_t*>(&b2);
-              pk[e] = u;
-              if (e & 1) add_bf16x2(lsum2, lsum3, u);
-              else add_bf16x2(lsum0, lsum1, u);
+            for (int c = 0; c < HALF / CH; ++c) {
+              const int k0 = hf * HALF + c * CH;
+              uint32_t pk[CH / 2];
+#pragma unroll
+              for (int e = 0; e < CH / 2; ++e) {
+                float p0, p1;
+                exp2_pair(s[k0 + 2 * e], s[k0 + 2 * e + 1], sl2, m_ref, sl2x2, negm2, emulated_pair(e), p0, p1);
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+                const uint32_t u = *reinterpret_cast<const uint32_t*>(&b2);
+                pk[e] = u;
+                if (e & 1) add_bf16x2(lsum2, lsum3, u);
+                else add_bf16x2(lsum0, lsum1, u);
+              }
+              if constexpr (CH == 64) tmem_st32(tS + k0 / 2, pk);
+              else tmem_st16(tS + k0 / 2, pk);
             }
-            tmem_st32(tS + c * 32, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(p_full + 2 * mt + hf);
           }
         } else {
           // P = hi + lo, both e4m3: the residual plane keeps the weights' relative
@@ -713,6 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // [0, BLK/4), lo in [BLK/4, BLK/2); packed 32 values (8 columns) at a time.
 #pragma unroll
           for (int c = 0; c < BLK / 32; ++c) {
+            const int hf = c / (BLK / 64);
             uint32_t phi[8], plo[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -739,12 +766,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tmem_st8(tS + 8 * c, phi);
             tmem_st8(tS + BLK / 4 + 8 * c, plo);
+            if (c % (BLK / 64) == BLK / 64 - 1) {  // last chunk of a half
+              tmem_wait_st();
+              tc_fence_before();
+              mbar_arrive(p_full + 2 * mt + hf);
+            }
           }
         }
         l += (lsum0 + lsum1) + (lsum2 + lsum3);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(p_full + mt);
       }
       if (!ok) break;
       // epilogue: O / l -> bf16, natural-log LSE

@@ -40,6 +40,9 @@ constexpr int kPoolThreads = 256;
 #define FP_POOL_UNROLL 4
 #endif
 constexpr int kPoolUnroll = FP_POOL_UNROLL;
+#ifndef FP_POOL_PIPE
+#define FP_POOL_PIPE 1
+#endif
 
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 v;
@@ -146,8 +149,42 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geometry g, const ui
     return isK ? (long long)qoff + t : (long long)qoff + t - p0;
   };
 
-  // kPoolUnroll independent 16-byte loads in flight per thread
   int t = t0 + p;
+#if FP_POOL_PIPE
+  // two batches of kPoolUnroll 16-byte loads: the next batch is in flight
+  // while the current one is accumulated
+  {
+    constexpr int U = kPoolUnroll;
+    const int step = U * tpi;
+    uint4 xa[U], xb[U];
+    auto full = [&](int tt) { return tt + (U - 1) * tpi < t1; };
+    auto load = [&](uint4* x, int tt) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const long long row = row_of(tt + u * tpi);
+        x[u] = row >= 0 ? ld_stream(base + row * row_bytes + head_off) : make_uint4(0, 0, 0, 0);
+      }
+    };
+    if (full(t)) {
+      load(xa, t);
+      for (;;) {
+        const bool nb = full(t + step);
+        if (nb) load(xb, t + step);
+#pragma unroll
+        for (int u = 0; u < U; ++u) accumulate<FP8>(acc, xa[u]);
+        t += step;
+        if (!nb) break;
+        const bool na = full(t + step);
+        if (na) load(xa, t + step);
+#pragma unroll
+        for (int u = 0; u < U; ++u) accumulate<FP8>(acc, xb[u]);
+        t += step;
+        if (!na) break;
+      }
+    }
+  }
+#else
+  // kPoolUnroll independent 16-byte loads in flight per thread
   for (; t + (kPoolUnroll - 1) * tpi < t1; t += kPoolUnroll * tpi) {
     uint4 x[kPoolUnroll];
 #pragma unroll
@@ -158,6 +195,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geometry g, const ui
 #pragma unroll
     for (int u = 0; u < kPoolUnroll; ++u) accumulate<FP8>(acc, x[u]);
   }
+#endif
   for (; t < t1; t += tpi) {
     const long long row = row_of(t);
     if (row >= 0) accumulate<FP8>(acc, ld_stream(base + row * row_bytes + head_off));

@@ -239,6 +239,7 @@ def check_attention(dev: Device, orc_out: dict, fp8: bool, report: dict | None =
             lse_err = max(lse_err, float(np.abs(gl - l).max()))
     mx = max(errs)
     mean = tot / n
+    print(f"attention {'e4m3' if fp8 else 'bf16'}: max abs {mx:.3e}, mean abs {mean:.3e}, lse {lse_err:.3e}")
     if report is not None:
         report.update(max_abs=mx, mean_abs=mean, lse_max_abs=lse_err)
     if fp8:
