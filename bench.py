@@ -98,7 +98,20 @@ class ClockSampler:
         except Exception:
             self.sel = str(device_index)
 
+    @staticmethod
+    def _rows(path):
+        rows = []
+        with open(path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        return rows
+
     def start(self):
+        """Starts sampling every 100 ms and returns once the first sample is in
+        (nvidia-smi takes a moment to start), so the timed region is covered."""
+        self.skip = 0
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
@@ -107,23 +120,28 @@ class ClockSampler:
                  "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, ValueError):
             self.proc = None
+            return
+        t0 = time.time()
+        while time.time() - t0 < 5.0 and self.proc.poll() is None:
+            n = len(self._rows(self.path))
+            if n:
+                self.skip = n  # samples taken before the timed region
+                return
+            time.sleep(0.02)
 
     def stop(self):
+        """Samples taken from the start of the timed region (at least one)."""
         if self.proc is None:
             return None
-        time.sleep(0.25)
+        time.sleep(0.15)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
+        rows = self._rows(self.path)
         os.unlink(self.path)
+        rows = rows[self.skip:] if len(rows) > self.skip else rows[-1:]
         if not rows:
             return None
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
