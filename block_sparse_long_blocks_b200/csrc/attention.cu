@@ -790,22 +790,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++on;
       tc_fence_after();
       const float inv = l > 0.f ? vmul / l : 0.f;  // a row that saw no key (masked everywhere) gets O = 0
+      // the O row in two TMEM round trips of 64 columns
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r32[32];
-        tmem_ld32(tO + c * 32, r32);
+      for (int hc = 0; hc < 2; ++hc) {
+        uint32_t r[64];
+        tmem_ld32(tO + hc * 64, r);
+        tmem_ld32(tO + hc * 64 + 32, r + 32);
         tmem_wait_ld();
         if (valid) {
-          uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r32[2 * e]) * inv,
-                                                            __uint_as_float(r32[2 * e + 1]) * inv);
-            pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
+          for (int c = 0; c < 8; ++c) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[8 * c + 2 * e]) * inv,
+                                                              __uint_as_float(r[8 * c + 2 * e + 1]) * inv);
+              pk[e] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            reinterpret_cast<uint4*>(orow_ptr + hc * 64)[c] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
-          uint4* dst = reinterpret_cast<uint4*>(orow_ptr + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         }
       }
       if (valid && a.lse)
