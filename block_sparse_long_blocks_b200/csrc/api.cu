@@ -116,13 +116,13 @@ Geometry geometry(const fp_params_t* p) {
   g.k_scale = p->k_scale;
   g.v_scale = p->v_scale;
   g.head_bits = p->head_bits;
-  g.attn_queue = nullptr;
   g.status = nullptr;
   return g;
 }
 
-// Workspace: pooled query planes, pooled key planes (256-byte aligned), then
-// the attention work-queue counter.
+// Workspace: pooled query planes, pooled key planes (256-byte aligned), the
+// attention work-queue counter (256 bytes), then the attention's claim order
+// (one int per work unit; fp_prefill only).
 size_t pad256(size_t bytes) { return (bytes + 255) / 256 * 256; }
 size_t pooled_q_bytes(const Geometry& g) { return pad256(3 * pooled_q_elems(g) * sizeof(__nv_bfloat16)); }
 size_t pooled_k_bytes(const Geometry& g) { return pad256(3 * pooled_k_elems(g) * sizeof(__nv_bfloat16)); }
@@ -130,9 +130,10 @@ size_t pooled_k_bytes(const Geometry& g) { return pad256(3 * pooled_k_elems(g) *
 int* queue_slot(const Geometry& g, void* ws) {
   return reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + pooled_q_bytes(g) + pooled_k_bytes(g));
 }
+int* order_slot(const Geometry& g, void* ws) { return queue_slot(g, ws) + 64; }
 
 fp_status_t discover_impl(const fp_params_t* p, const void* q, const void* k, uint32_t* mask, int32_t* idx,
-                          int32_t* cnt, void* ws, size_t ws_bytes, void* stream, bool zero_queue = false) {
+                          int32_t* cnt, void* ws, size_t ws_bytes, void* stream) {
   fp_status_t st = validate(p, false);
   if (st != FP_OK) return st;
   if (!q || !k || (!mask && !idx) || (idx && !cnt)) return FP_ERR_INVALID_ARG;
@@ -144,7 +145,6 @@ fp_status_t discover_impl(const fp_params_t* p, const void* q, const void* k, ui
   Geometry g = geometry(p);
   g.status = status_ptr();
   if (!g.status) return cuda_fail("device status symbol", cudaGetLastError());
-  if (zero_queue) g.attn_queue = queue_slot(g, ws);
   __nv_bfloat16* qpl = static_cast<__nv_bfloat16*>(ws);
   __nv_bfloat16* kpl = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + pooled_q_bytes(g));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -165,7 +165,7 @@ fp_status_t attention_impl(const fp_params_t* p, bool paged, const void* q, cons
   Geometry g = geometry(p);
   g.status = status_ptr();
   if (!g.status) return cuda_fail("device status symbol", cudaGetLastError());
-  return launch_attention(g, q, k, v, idx, cnt, o, lse, static_cast<cudaStream_t>(stream), nullptr, false);
+  return launch_attention(g, q, k, v, idx, cnt, o, lse, static_cast<cudaStream_t>(stream), nullptr, nullptr, false);
 }
 
 }  // namespace
@@ -178,7 +178,8 @@ extern "C" {
 size_t fp_workspace_size(const fp_params_t* p) {
   if (validate(p, false) != FP_OK) return 0;
   const Geometry g = geometry(p);
-  return pooled_q_bytes(g) + pooled_k_bytes(g) + 256;  // + work-queue counter
+  // + work-queue counter + claim order (when the attention supports this geometry)
+  return pooled_q_bytes(g) + pooled_k_bytes(g) + 256 + pad256((size_t)attention_units(g) * sizeof(int));
 }
 
 size_t fp_mask_words(const fp_params_t* p) {
@@ -241,11 +242,16 @@ fp_status_t fp_prefill(const fp_params_t* p, const void* q, const void* k, const
   if (st != FP_OK) return st;
   if (!v || !o) return FP_ERR_INVALID_ARG;
   if (!aligned(v, 16) || !aligned(o, 16) || (lse && !aligned(lse, 4))) return FP_ERR_ALIGNMENT;
-  st = discover_impl(p, q, k, mask, idx, cnt, workspace, ws_bytes, stream, /*zero_queue=*/true);
+  if (!idx || !cnt) return FP_ERR_INVALID_ARG;
+  st = discover_impl(p, q, k, mask, idx, cnt, workspace, ws_bytes, stream);
   if (st != FP_OK) return st;
   Geometry g = geometry(p);
   g.status = status_ptr();
-  return launch_attention(g, q, k, v, idx, cnt, o, lse, static_cast<cudaStream_t>(stream), queue_slot(g, workspace),
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // longest lists first: the claim order of the attention's device queue
+  const cudaError_t e = launch_unit_order(g, cnt, order_slot(g, workspace), queue_slot(g, workspace), s);
+  if (e != cudaSuccess) return cuda_fail("unit order launch", e);
+  return launch_attention(g, q, k, v, idx, cnt, o, lse, s, queue_slot(g, workspace), order_slot(g, workspace),
                           /*pdl=*/true);
 }
 

@@ -208,7 +208,8 @@ struct AttnArgs {
   const int32_t* cnt;
   __nv_bfloat16* o;
   float* lse;
-  int* queue;  // device work-queue counter (zeroed before launch) or nullptr: static schedule
+  int* queue;          // device work-queue counter (zeroed before launch) or nullptr: static schedule
+  const int* order;    // with a queue: the units in claim order (longest lists first)
 };
 
 template <bool FP8, int BLK>
@@ -240,17 +241,20 @@ struct Cfg {
 };
 
 // Work units reach the roles either by a static stride over the persistent
-// grid or, with a device queue, in claim order: the producer claims each unit
-// (atomicAdd on the queue) and passes it to the MMA and softmax roles through
-// a small ring in shared memory guarded by full/empty mbarriers.
+// grid or, with a device queue, in claim order: the producer claims the next
+// position (atomicAdd on the queue), looks the unit up in the longest-first
+// order and passes it to the MMA and softmax roles through a small ring in
+// shared memory guarded by full/empty mbarriers.
 struct UnitIter {
   int* queue;
+  const int* order;
   int* ring;
   uint64_t* full;
   uint64_t* empty;
   volatile int* abort;
   unsigned* status;
   bool producer;
+  long long num_units;
   long long u;
   int n;
 
@@ -267,7 +271,8 @@ struct UnitIter {
         ok = false;
         return LLONG_MAX;
       }
-      const int v = atomicAdd(queue, 1);
+      int v = atomicAdd(queue, 1);
+      if (v < num_units) v = __ldg(order + v);
       ring[slot] = v;
       mbar_arrive(full + slot);
       return v;
@@ -443,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       long long kt = 0, vt = 0, qn = 0;
       const uint32_t q_bytes = 2u * C::DCH * a.rows * 128u;
       bool ok = true;
-      UnitIter it{a.queue, unit_ring, unit_full, unit_empty, abort_flag, g.status, true, 0, 0};
+      UnitIter it{a.queue, a.order, unit_ring, unit_full, unit_empty, abort_flag, g.status, true, a.num_units, 0, 0};
       for (long long u = it.step(true, ok); u < a.num_units && ok; u = it.step(false, ok)) {
         Unit U;
         if (!decode_unit(u, a, U) || U.count == 0) continue;
@@ -531,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
 
-      UnitIter it{a.queue, unit_ring, unit_full, unit_empty, abort_flag, g.status, false, 0, 0};
+      UnitIter it{a.queue, a.order, unit_ring, unit_full, unit_empty, abort_flag, g.status, false, a.num_units, 0, 0};
       for (long long u = it.step(true, ok); u < a.num_units && ok; u = it.step(false, ok)) {
         Unit U;
         if (!decode_unit(u, a, U) || U.count == 0) continue;
@@ -614,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int hh = row % g.G, tt = row / g.G;
     long long sn = 0, on = 0;
     bool ok = true;
-    UnitIter it{a.queue, unit_ring, unit_full, unit_empty, abort_flag, g.status, false, 0, 0};
+    UnitIter it{a.queue, a.order, unit_ring, unit_full, unit_empty, abort_flag, g.status, false, a.num_units, 0, 0};
     for (long long u = it.step(true, ok); u < a.num_units && ok; u = it.step(false, ok)) {
       Unit U;
       if (!decode_unit(u, a, U)) continue;
@@ -894,20 +899,107 @@ fp_status_t run(const AttnArgs& a, const void* q, const void* k, const void* v, 
 
 }  // namespace
 
-fp_status_t launch_attention(const Geometry& g, const void* q, const void* k, const void* v, const int32_t* idx,
-                             const int32_t* cnt, void* o, float* lse, cudaStream_t s, int* queue, bool pdl) {
-  AttnArgs a;
-  a.queue = queue;
-  a.g = g;
-  int Tm = 1;
+// Tokens per M-tile (Tm), M-tile pairs per query block and work units of the
+// attention for this geometry; false when B / Tm is not an even number >= 2.
+bool attention_layout(const Geometry& g, int& Tm, int& nPairs, long long& units) {
+  Tm = 1;
   while (Tm * 2 * g.G <= 128 && Tm * 2 <= g.B) Tm *= 2;
   const int nM = g.B / Tm;
-  if (nM < 2 || nM % 2 != 0) return FP_ERR_UNSUPPORTED;
-  if ((long long)g.Nmax * g.R * g.Hkv * (nM / 2) >= INT_MAX) return FP_ERR_UNSUPPORTED;  // int unit ids
+  if (nM < 2 || nM % 2 != 0) return false;
+  nPairs = nM / 2;
+  units = (long long)g.Nmax * g.R * g.Hkv * nPairs;
+  return true;
+}
+
+long long attention_units(const Geometry& g) {
+  int Tm, nPairs;
+  long long units;
+  return attention_layout(g, Tm, nPairs, units) ? units : 0;
+}
+
+namespace {
+
+constexpr int kOrderThreads = 1024;
+
+// Claim order for the device work queue, longest lists first: the work units
+// sorted by their row's list length, descending (a counting sort over the
+// lengths 0..Nmax; the M-tile pairs of one row stay together, rows of equal
+// length in arbitrary order). One CTA; it also zeroes the queue counter.
+__global__ void __launch_bounds__(kOrderThreads)
+    unit_order_kernel(const Geometry g, int nPairs, const int32_t* __restrict__ cnt, int* __restrict__ order,
+                      int* __restrict__ queue) {
+  // the attention, launched as a programmatic dependent, may start its prologue
+  asm volatile("griddepcontrol.launch_dependents;");
+  extern __shared__ int start[];  // [Nmax + 1]: rows per length, then first unit position per length
+  __shared__ int warp_tot[kOrderThreads / 32];
+  const int bins = g.Nmax + 1;
+  const long long rows = (long long)g.R * g.Hkv * g.Nmax;
+  auto key = [&](long long row) {
+    const int c = __ldg(cnt + row);
+    return c < 0 ? 0 : (c > g.Nmax ? g.Nmax : c);
+  };
+  for (int b = threadIdx.x; b < bins; b += kOrderThreads) start[b] = 0;
+  if (threadIdx.x == 0) *queue = 0;
+  __syncthreads();
+  for (long long row = threadIdx.x; row < rows; row += kOrderThreads) atomicAdd(&start[key(row)], 1);
+  __syncthreads();
+  // exclusive prefix over the lengths in descending order (thread t owns a run of them)
+  const int per = (bins + kOrderThreads - 1) / kOrderThreads;
+  const int d0 = threadIdx.x * per, d1 = min(d0 + per, bins);
+  int local = 0;
+  for (int d = d0; d < d1; ++d) local += start[bins - 1 - d];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  int before = 0;
+  for (int w = 0; w < warp; ++w) before += warp_tot[w];
+  int run = before + incl - local;  // rows of longer lists
+  for (int d = d0; d < d1; ++d) {
+    const int b = bins - 1 - d, n = start[b];
+    start[b] = run * nPairs;
+    run += n;
+  }
+  __syncthreads();
+  const int RH = g.R * g.Hkv;
+  for (long long row = threadIdx.x; row < rows; row += kOrderThreads) {
+    const int pos = atomicAdd(&start[key(row)], nPairs);
+    const int i = (int)(row % g.Nmax), rk = (int)(row / g.Nmax);  // rk = r * Hkv + kvh
+    const int u0 = ((g.Nmax - 1 - i) * RH + rk) * nPairs;
+    for (int p = 0; p < nPairs; ++p) order[pos + p] = u0 + p;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_unit_order(const Geometry& g, const int32_t* cnt, int* order, int* queue, cudaStream_t s) {
+  int Tm, nPairs;
+  long long units;
+  if (!attention_layout(g, Tm, nPairs, units)) return cudaErrorInvalidValue;
+  unit_order_kernel<<<1, kOrderThreads, (size_t)(g.Nmax + 1) * sizeof(int), s>>>(g, nPairs, cnt, order, queue);
+  return cudaGetLastError();
+}
+
+fp_status_t launch_attention(const Geometry& g, const void* q, const void* k, const void* v, const int32_t* idx,
+                             const int32_t* cnt, void* o, float* lse, cudaStream_t s, int* queue, const int* order,
+                             bool pdl) {
+  AttnArgs a;
+  a.queue = queue;
+  a.order = order;
+  a.g = g;
+  int Tm, nPairs;
+  long long units;
+  if (!attention_layout(g, Tm, nPairs, units)) return FP_ERR_UNSUPPORTED;
+  if (units >= INT_MAX) return FP_ERR_UNSUPPORTED;  // int unit ids
   a.Tm = Tm;
   a.rows = Tm * g.G;
-  a.nPairs = nM / 2;
-  a.num_units = (long long)g.Nmax * g.R * g.Hkv * a.nPairs;
+  a.nPairs = nPairs;
+  a.num_units = units;
   a.T = g.cu ? (long long)g.total_tokens : (long long)g.R * g.L;
   a.scale_log2 = g.scale * 1.4426950408889634f;
   a.idx = idx;

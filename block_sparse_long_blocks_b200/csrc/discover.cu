@@ -292,9 +292,6 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kScoreBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  // a following programmatic-dependent launch (the attention) may start its prologue
-  asm volatile("griddepcontrol.launch_dependents;");
-  if (blockIdx.x == 0 && threadIdx.x == 0 && g.attn_queue) *g.attn_queue = 0;
 
   const int RH = g.R * g.Hkv;
   const int tiles = (g.Nmax + QB - 1) / QB;

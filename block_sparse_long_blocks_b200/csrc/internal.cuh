@@ -31,7 +31,6 @@ struct Geometry {
   const float* k_scale;
   const float* v_scale;
   uint8_t* head_bits;       // per-head selection bits per list entry, or nullptr
-  int* attn_queue;          // discovery zeroes this attention work-queue counter, or nullptr
   unsigned* status;         // device status word
 };
 
@@ -96,10 +95,16 @@ cudaError_t launch_compact(const Geometry& g, const uint32_t* mask, int32_t* idx
                            cudaStream_t s);
 // Returns FP_OK, FP_ERR_UNSUPPORTED or FP_ERR_CUDA.
 // queue: zeroed device counter for claim-order scheduling, or nullptr (static
-// stride). pdl: launch as a programmatic dependent of the previous kernel.
+// stride); order: the units in claim order (launch_unit_order). pdl: launch as
+// a programmatic dependent of the previous kernel.
 fp_status_t launch_attention(const Geometry& g, const void* q, const void* k, const void* v,
                              const int32_t* idx, const int32_t* cnt, void* o, float* lse,
-                             cudaStream_t s, int* queue, bool pdl);
+                             cudaStream_t s, int* queue, const int* order, bool pdl);
+// Attention work units of this geometry (0 when the attention does not support it).
+long long attention_units(const Geometry& g);
+// Writes the attention's longest-first claim order (attention_units(g) ints)
+// from the list lengths and zeroes the queue counter.
+cudaError_t launch_unit_order(const Geometry& g, const int32_t* cnt, int* order, int* queue, cudaStream_t s);
 
 // cuTensorMapEncodeTiled (through the runtime's driver entry point) with
 // 128-byte swizzle, 256-byte L2 promotion and zero fill outside the tensor.

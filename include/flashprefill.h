@@ -122,8 +122,9 @@ typedef struct {
 } fp_params_t;
 
 /* Bytes of device scratch fp_discover needs: the pooled Q and K, each pooled
- * float32 value stored as three bf16 parts (hi + mid + lo), plus 256 bytes
- * for fp_prefill's work-queue counter. */
+ * float32 value stored as three bf16 parts (hi + mid + lo), plus what
+ * fp_prefill adds: a work-queue counter (256 bytes) and the attention's claim
+ * order (one int per work unit). */
 size_t fp_workspace_size(const fp_params_t* p);
 /* Number of uint32 words of the block mask: R * Hkv * Nmax * ceil(Nmax / 32). */
 size_t fp_mask_words(const fp_params_t* p);
@@ -188,12 +189,13 @@ fp_status_t fp_paged_sparse_prefill(const fp_params_t* p, const void* q, const v
  * The whole path in one call: discovery + compaction (as fp_discover_compact,
  * mask may be NULL) followed by the block-sparse attention (as
  * fp_sparse_prefill, or fp_paged_sparse_prefill when p->page_table is set;
- * k and v are then the pools). The attention is launched as a programmatic
- * dependent of the discovery, so its prologue overlaps discovery's tail, and
- * it takes its work units (request, KV group, query block, M-tile pair) from
- * a device queue in the workspace, longest query blocks first, instead of a
- * static stride. workspace: fp_workspace_size(p) bytes as for fp_discover.
- * Outputs are identical to the three separate calls.
+ * k and v are then the pools). Between the two a one-CTA kernel sorts the
+ * attention's work units (request, KV group, query block, M-tile pair) by
+ * their list length, longest first; the attention is launched as a
+ * programmatic dependent of it, so its prologue overlaps the sort, and claims
+ * the units in that order from a device queue in the workspace instead of a
+ * static stride. idx and cnt are required. workspace: fp_workspace_size(p)
+ * bytes as for fp_discover. Outputs are identical to the three separate calls.
  */
 fp_status_t fp_prefill(const fp_params_t* p, const void* q, const void* k, const void* v, uint32_t* mask,
                        int32_t* idx, int32_t* cnt, void* o, float* lse, void* workspace, size_t ws_bytes,
