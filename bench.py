@@ -544,6 +544,12 @@ def short_context(setup, stream):
 
 
 def e2e(args, D, inp_host, dev, stream, dense, world, dist):
+    """The metric end to end through the C ABI: every step copies its Q/K/V in
+    from pinned host memory, runs discovery + compaction + attention and
+    copies O back. Steps are pipelined over two device buffer sets on three
+    streams (inputs of step n+1 and the output of step n-1 cross PCIe while
+    step n computes), as a serving loop would; the timed region runs from the
+    first input copy to the last output copy."""
     from block_sparse_long_blocks_b200 import binding as fb
     paged = D["paged"]
     hq = inp_host.q.pin_memory()
@@ -552,32 +558,52 @@ def e2e(args, D, inp_host, dev, stream, dense, world, dist):
     ho = torch.empty(tuple(inp_host.q.shape), dtype=torch.bfloat16).pin_memory()
     h2d = hq.numel() * hq.element_size() + hk.numel() * hk.element_size() + hv.numel() * hv.element_size()
     d2h = ho.numel() * ho.element_size()
-    steps = max(3, min(args.steps, 5))
+    steps = max(3, min(args.steps, 8))
+    sets = [dict(q=D["q"], k=D["k"], v=D["v"], o=D["bufs"].o, ws=D["bufs"].workspace, idx=D["bufs"].idx,
+                 cnt=D["bufs"].cnt)]
+    sets.append({n: torch.empty_like(t) for n, t in sets[0].items()})
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    h2d_done, cmp_done, d2h_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    for e in cmp_done + d2h_done:
+        e.record(stream)
 
-    def one():
-        D["q"].copy_(hq, non_blocking=True)
-        D["k"].copy_(hk, non_blocking=True)
-        D["v"].copy_(hv, non_blocking=True)
-        fb.fp_discover_compact(D["p"], D["q"], D["k"], None, D["bufs"].idx, D["bufs"].cnt, D["bufs"].workspace)
+    def one(n):
+        b = sets[n % 2]
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(cmp_done[n % 2])  # step n-2 is done reading this set
+            b["q"].copy_(hq, non_blocking=True)
+            b["k"].copy_(hk, non_blocking=True)
+            b["v"].copy_(hv, non_blocking=True)
+            h2d_done[n % 2].record(s_in)
+        stream.wait_event(h2d_done[n % 2])
+        stream.wait_event(d2h_done[n % 2])  # step n-2's output has left this set
+        fb.fp_discover_compact(D["p"], b["q"], b["k"], None, b["idx"], b["cnt"], b["ws"])
         if paged:
-            fb.fp_paged_sparse_prefill(D["p"], D["q"], D["k"], D["v"], D["bufs"].idx, D["bufs"].cnt, D["bufs"].o)
+            fb.fp_paged_sparse_prefill(D["p"], b["q"], b["k"], b["v"], b["idx"], b["cnt"], b["o"])
         else:
-            fb.fp_sparse_prefill(D["p"], D["q"], D["k"], D["v"], D["bufs"].idx, D["bufs"].cnt, D["bufs"].o)
-        ho.copy_(D["bufs"].o, non_blocking=True)
+            fb.fp_sparse_prefill(D["p"], b["q"], b["k"], b["v"], b["idx"], b["cnt"], b["o"])
+        cmp_done[n % 2].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(cmp_done[n % 2])
+            ho.copy_(b["o"], non_blocking=True)
+            d2h_done[n % 2].record(s_out)
 
-    one()
+    one(0)
+    one(1)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist is not None:
         dist.barrier()
-    a.record(stream)
-    for _ in range(steps):
-        one()
-    b.record(stream)
+    a.record(s_in)
+    for n in range(steps):
+        one(n)
+    b.record(s_out)
     torch.cuda.synchronize()
     ms = max_over_ranks([a.elapsed_time(b) / steps], dist, dev)[0]
     return {"value": weak_value(world, dense, ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps,
+            "pipelined": "two buffer sets, inputs / compute / output on three streams"}
 
 
 def fp8_extra(args, w, inp_host, dev, stream, pk, setup, dist):

@@ -80,7 +80,7 @@ fp_status_t validate(const fp_params_t* p, bool attention) {
   }
   if (attention) {
     int Tm = 1;
-    while (Tm * 2 * G <= 128 && Tm * 2 <= p->block) Tm *= 2;
+    while (Tm * 2 * G <= 128 && Tm * 2 <= p->block / 2) Tm *= 2;  // >= 2 M-tiles per query block
     if (p->block / Tm < 2) return FP_ERR_UNSUPPORTED;
   }
   return FP_OK;

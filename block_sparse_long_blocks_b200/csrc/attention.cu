@@ -8,8 +8,8 @@
 // Work unit = (request r, KV group kvh, query block i, M-tile pair). PackGQA:
 // the rows of an M-tile are (token, head) pairs of one KV group, token-major
 // (row = t * G + h), Tm tokens x G heads with Tm the largest power of two such
-// that Tm * G <= 128, so every K/V tile a CTA loads serves all G heads. A CTA
-// owns two M-tiles (ping-pong) and walks row (r, kvh, i)'s list.
+// that Tm * G <= 128 and Tm <= B / 2, so every K/V tile a CTA loads serves all
+// G heads. A CTA owns two M-tiles (ping-pong) and walks row (r, kvh, i)'s list.
 //
 // Roles (384 threads, one persistent CTA per SM):
 //   warps 0-3  softmax warpgroup for M-tile 0 (one thread per row)
@@ -640,7 +640,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool last_is_diag = U.count > 0 && __ldg(a.idx + U.lbase + U.count - 1) == U.i;
       // per-head selection: a visited block this row's head did not keep is masked
       const uint8_t* hbp = g.head_bits ? g.head_bits + U.lbase : nullptr;
-      uint32_t hb_next = (hbp && U.count > 0) ? __ldg(hbp) : 0xFFu;
+      // (without head bits every head keeps every listed block, G up to 16)
+      uint32_t hb_next = (hbp && U.count > 0) ? __ldg(hbp) : 0xFFFFFFFFu;
       for (int n = 0; n < U.count; ++n) {
         const uint32_t hb = hb_next;
         if (hbp && n + 1 < U.count) hb_next = __ldg(hbp + n + 1);  // one visit ahead
@@ -903,7 +904,9 @@ fp_status_t run(const AttnArgs& a, const void* q, const void* k, const void* v, 
 // attention for this geometry; false when B / Tm is not an even number >= 2.
 bool attention_layout(const Geometry& g, int& Tm, int& nPairs, long long& units) {
   Tm = 1;
-  while (Tm * 2 * g.G <= 128 && Tm * 2 <= g.B) Tm *= 2;
+  // at least two M-tiles per query block (a work unit is a pair of them): for
+  // G = 1 at B = 128, or G <= 2 at B = 64, the M-tiles are half full
+  while (Tm * 2 * g.G <= 128 && Tm * 2 <= g.B / 2) Tm *= 2;
   const int nM = g.B / Tm;
   if (nM < 2 || nM % 2 != 0) return false;
   nPairs = nM / 2;

@@ -139,6 +139,30 @@ def test_attention_on_oracle_lists(name, L, alpha, fp8):
     H.check_attention(dev, H.oracle_attention(w, inp, orc), fp8)
 
 
+# PackGQA M-tile shapes beyond G = 4, 7, 8: G = 1 (64 tokens x 1 head, one
+# M-tile pair per block), G = 3 (32 x 3 = 96 rows), G = 16 (8 x 16 = 128 rows,
+# eight pairs per block), and G = 2 at block 64 (32 x 2).
+GROUP_CASES = [
+    ("qwen30b_128k", 2600, {"hq": 4}),
+    ("qwen30b_128k", 2600, {"hq": 6, "hkv": 2}),
+    ("qwen30b_128k", 2600, {"hkv": 2}),
+    ("tiny2k", 1500, {"hq": 2}),
+]
+
+
+@pytest.mark.parametrize("name,L,kw", GROUP_CASES)
+@pytest.mark.parametrize("fp8", [False, True])
+def test_attention_group_shapes(name, L, kw, fp8):
+    w = _case(name, L, **kw)
+    inp = _inputs(w, fp8)
+    dev = H.Device(w, inp)
+    orc = H.oracle_discovery(w, inp)
+    idx, cnt = H.upload_lists(dev.cfg, [o["lists"] for o in orc])
+    dev.attend(idx, cnt)
+    assert dev.status() == 0
+    H.check_attention(dev, H.oracle_attention(w, inp, orc), fp8)
+
+
 @pytest.mark.parametrize("fp8", [False, True])
 def test_full_path_tiny(fp8):
     """Discovery -> compaction -> attention on the GPU; lists equal the oracle's."""
