@@ -34,15 +34,12 @@ namespace fp {
 namespace {
 
 constexpr int kPoolThreads = 256;
-// Loads in flight per pooling thread. 4 measured best: 8 costs occupancy
-// (registers) and lowers the achieved bandwidth.
+// Loads per batch of a pooling thread (two batches in flight). 4 measured
+// best: 8 costs occupancy (registers) and lowers the achieved bandwidth.
 #ifndef FP_POOL_UNROLL
 #define FP_POOL_UNROLL 4
 #endif
 constexpr int kPoolUnroll = FP_POOL_UNROLL;
-#ifndef FP_POOL_PIPE
-#define FP_POOL_PIPE 1
-#endif
 
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 v;
@@ -150,7 +147,6 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geometry g, const ui
   };
 
   int t = t0 + p;
-#if FP_POOL_PIPE
   // two batches of kPoolUnroll 16-byte loads: the next batch is in flight
   // while the current one is accumulated
   {
@@ -183,19 +179,6 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geometry g, const ui
       }
     }
   }
-#else
-  // kPoolUnroll independent 16-byte loads in flight per thread
-  for (; t + (kPoolUnroll - 1) * tpi < t1; t += kPoolUnroll * tpi) {
-    uint4 x[kPoolUnroll];
-#pragma unroll
-    for (int u = 0; u < kPoolUnroll; ++u) {
-      const long long row = row_of(t + u * tpi);
-      x[u] = row >= 0 ? ld_stream(base + row * row_bytes + head_off) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < kPoolUnroll; ++u) accumulate<FP8>(acc, x[u]);
-  }
-#endif
   for (; t < t1; t += tpi) {
     const long long row = row_of(t);
     if (row >= 0) accumulate<FP8>(acc, ld_stream(base + row * row_bytes + head_off));
