@@ -55,6 +55,37 @@ def test_buffer_sizes(lib):
     assert s["mask_words"] == 3 * 4 * N * 1 and s["count_entries"] == 3 * 4 * N
 
 
+def _pad256(n):
+    return (n + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("kw,pairs", [({}, 4), (dict(hq=4), 1), (dict(hkv=2), 8), (dict(hq=6, hkv=2), 2)])
+def test_workspace_layout(lib, kw, pairs):
+    """Pooled query and key planes (three bf16 parts each), the work-queue
+    counter and the claim order of the attention's work units: M-tile pairs
+    per query block = B / (2 Tm), Tm the largest power of two with Tm G <= 128
+    and Tm <= B / 2."""
+    cfg = _cfg(**kw)
+    p = fb.make_params(cfg)
+    N, R, Hq, Hkv = cfg.nmax, cfg.batch, cfg.hq, cfg.hkv
+    q_planes = _pad256(3 * 2 * R * N * Hq * 128)
+    k_planes = _pad256(3 * 2 * R * Hkv * N * 128)
+    order = _pad256(4 * N * R * Hkv * pairs)
+    assert fb.sizes(p)["workspace"] == q_planes + k_planes + 256 + order
+
+
+def test_single_call_argument_checks(lib):
+    p = fb.make_params(_cfg())
+    ok = 1 << 20  # never dereferenced: validation fails first
+    ws = lib.fp_workspace_size(ctypes.byref(p))
+    f = lib.fp_prefill
+    assert f(ctypes.byref(p), ok, ok, ok, None, None, ok, ok, None, ok, ws, None) == -1   # idx missing
+    assert f(ctypes.byref(p), ok, ok, ok, None, ok, None, ok, None, ok, ws, None) == -1   # cnt missing
+    assert f(ctypes.byref(p), ok, ok, None, None, ok, ok, ok, None, ok, ws, None) == -1   # v missing
+    assert f(ctypes.byref(p), ok, ok, ok, None, ok, ok, ok + 8, None, ok, ws, None) == -3  # o misaligned
+    assert f(ctypes.byref(p), ok, ok, ok, None, ok, ok, ok, None, ok, ws - 1, None) == -4  # workspace short
+
+
 @pytest.mark.parametrize("bad,code", [
     (dict(head_dim=64), -2), (dict(block=32), -2), (dict(alpha=-0.5), -1), (dict(alpha=float("nan")), -1),
     (dict(alpha=float("inf")), -1), (dict(hq=30, hkv=4), -1), (dict(batch=0), -1), (dict(max_seqlen=0), -1),
