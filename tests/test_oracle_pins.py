@@ -511,3 +511,20 @@ def test_per_head_attention_equals_per_head_masked_sdpa(alpha):
     v = torch.from_numpy(np.repeat(V, hq // hkv, axis=1)).permute(1, 0, 2)[None]
     want = F.scaled_dot_product_attention(q, k, v, attn_mask=torch.from_numpy(tm)[None], scale=r["scale"])
     np.testing.assert_allclose(O, want[0].permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_row_borderline_finds_blocks_at_alpha():
+    """Pooled vectors built so that block 1 has exactly probability alpha in
+    head 0's row and block 2 sits well above it: only block 1 is borderline,
+    and a perturbation beyond the band takes it out."""
+    alpha, scale, d = 0.1, 1.0, 4
+    kbar = np.zeros((3, 1, d))
+    kbar[0, 0, 0] = 1.0                    # s0 = 1 (row max)
+    kbar[1, 0, 0] = 1.0 + math.log(alpha)  # s1 - s0 = ln(alpha): p1 = alpha exactly
+    kbar[2, 0, 0] = 0.9                    # p2 = exp(-0.1), far from alpha
+    qbar = np.zeros((3, 1, d))
+    qbar[2, 0, 0] = 1.0
+    assert fo.row_borderline(qbar, kbar, scale, alpha, 0, 2) == {1}
+    kbar[1, 0, 0] += 1e-3                  # p1 = alpha * e^1e-3: outside 1e-5 relative
+    assert fo.row_borderline(qbar, kbar, scale, alpha, 0, 2) == set()
+    assert fo.row_borderline(qbar, kbar, scale, 0.0, 0, 2) == set()  # alpha = 0 has no boundary
