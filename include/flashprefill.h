@@ -114,7 +114,7 @@ typedef struct {
   const int32_t* cu_seqlens;  /* device int32 [batch + 1] or NULL (contiguous batch) */
   int total_tokens;           /* varlen: cu_seqlens[batch] (rows of the packed Q) */
   const int32_t* page_table;  /* device int32 [batch, max_pages_per_req] or NULL */
-  int page_size;              /* paged: tokens per page (power of two, 16..256) */
+  int page_size;              /* paged: tokens per page (power of two, 16..65536) */
   int max_pages_per_req;
   int num_pages;              /* paged: pages in each pool */
   const int32_t* kv_lens;     /* chunked prefill: device int32 [batch] or NULL (see below) */
