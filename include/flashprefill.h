@@ -82,7 +82,9 @@ extern "C" {
 typedef enum {
   FP_OK = 0,
   FP_ERR_INVALID_ARG = -1,  /* null pointer, bad size, alpha < 0 or not finite */
-  FP_ERR_UNSUPPORTED = -2,  /* head_dim != 128, block not 64/128, unsupported G */
+  FP_ERR_UNSUPPORTED = -2,  /* head_dim != 128, block not 64/128, G = hq / hkv not in
+                               1..8 or 16, Nmax > 8192, page size not a power of two in
+                               16..65536 */
   FP_ERR_ALIGNMENT = -3,    /* a tensor pointer is not 16-byte aligned */
   FP_ERR_WORKSPACE = -4,    /* workspace missing or smaller than fp_workspace_size */
   FP_ERR_CUDA = -5,         /* a CUDA runtime call or launch failed */
