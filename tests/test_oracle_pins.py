@@ -528,3 +528,22 @@ def test_row_borderline_finds_blocks_at_alpha():
     kbar[1, 0, 0] += 1e-3                  # p1 = alpha * e^1e-3: outside 1e-5 relative
     assert fo.row_borderline(qbar, kbar, scale, alpha, 0, 2) == set()
     assert fo.row_borderline(qbar, kbar, scale, 0.0, 0, 2) == set()  # alpha = 0 has no boundary
+
+
+# ----------------------------------------------------------------------------- randomised
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=40, deadline=None, derandomize=True)
+@given(L=st.integers(1, 40), B=st.sampled_from([4, 8, 16]), hkv=st.integers(1, 2), G=st.integers(1, 3),
+       alpha=st.sampled_from([0.0, 1e-3, 0.1, 0.5, 1.0, 2.0]), sink=st.integers(0, 12), win=st.integers(0, 20),
+       seed=st.integers(0, 10_000))
+def test_oracle_matches_brute_force_random_shapes(L, B, hkv, G, alpha, sink, win, seed):
+    """The vectorised oracle against the per-element brute force on random tiny
+    shapes (ragged tails, every group size up to 3, sink/window in tokens)."""
+    Q, K, V = _rand(L, hkv * G, hkv, 4, seed, amp=2.0 if L > 4 else 0.0)  # (heavy blocks need L > 4)
+    r = oracle.flashprefill(Q, K, V, B, alpha, sink, win)
+    bf = oracle.brute_force(Q.tolist(), K.tolist(), V.tolist(), B, alpha, sink, win)
+    assert _lists(r) == bf["lists"]
+    np.testing.assert_allclose(r["O"], np.array(bf["O"]), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(r["lse"], np.array(bf["lse"]), rtol=1e-10, atol=1e-12)
