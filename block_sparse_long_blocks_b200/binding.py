@@ -65,11 +65,9 @@ class Params(ctypes.Structure):
 _lib = None
 
 
-def load(path: str = LIB_PATH) -> ctypes.CDLL:
-    """Load the in-tree library (raises if it has not been built)."""
-    global _lib
-    if _lib is not None:
-        return _lib
+def load_library(path: str) -> ctypes.CDLL:
+    """A handle on a build of the library at ``path`` with every entry point's
+    signature declared (not cached: build variants load side by side)."""
     if not os.path.exists(path):
         raise RuntimeError(f"{path} is missing: build it with `python -m block_sparse_long_blocks_b200.build`")
     lib = ctypes.CDLL(path)
@@ -96,8 +94,15 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         f = getattr(lib, name)
         f.restype = res
         f.argtypes = args
-    _lib = lib
     return lib
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the in-tree library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        _lib = load_library(path)
+    return _lib
 
 
 @dataclass

@@ -105,58 +105,15 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 
-// 2^x for a pair of x <= 8 on the FMA pipe, to take load off the MUFU unit.
-// Cody-Waite style range reduction x = j + f: j = round(x) obtained by adding
-// 1.5*2^23 (the float then holds j in its low mantissa bits), f = x - j in
-// [-0.5, 0.5]; 2^f by a degree-3 polynomial whose coefficients were fitted for
-// minimum maximum relative error on [-0.5, 0.5] (7.5e-5, far below the bf16 /
-// e4m3 rounding that follows); 2^j by adding j to the exponent field. Inputs
-// are clamped at -125 so the exponent field stays normal (2^-125 stands in for
-// 0, which is negligible against a row maximum of at least 1).
-__device__ __forceinline__ void exp2_poly2(uint64_t x2, float& y0, float& y1) {
-  float x0, x1;
-  f2_unpack(x2, x0, x1);
-  x2 = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-  const float kMagic = 12582912.0f;  // 1.5 * 2^23
-  const uint64_t t2 = f2_add(x2, f2_pack(kMagic, kMagic));
-  const uint64_t r2 = f2_add(t2, f2_pack(-kMagic, -kMagic));
-  const uint64_t f2 = f2_fma(r2, f2_pack(-1.f, -1.f), x2);
-  uint64_t p2 = f2_fma(f2_pack(0.05517132207751274f, 0.05517132207751274f), f2,
-                       f2_pack(0.24261054396629333f, 0.24261054396629333f));
-  p2 = f2_fma(p2, f2, f2_pack(0.6932609677314758f, 0.6932609677314758f));
-  p2 = f2_fma(p2, f2, f2_pack(0.9999281167984009f, 0.9999281167984009f));
-  float p0, p1, t0, t1;
-  f2_unpack(p2, p0, p1);
-  f2_unpack(t2, t0, t1);
-  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
-// One pair of softmax weights 2^(s*sl2 - m): packed scale-and-subtract, then
-// every kEmuEvery-th pair on the FMA pipe and the rest on MUFU.EX2.
-// Tuning knobs (compile time): FP_EMU_EVERY = 0 disables the FMA-pipe exp2;
-// FP_PACKED_FMA selects the packed float32x2 scale-and-subtract.
-#ifndef FP_EMU_EVERY
-#define FP_EMU_EVERY 0
-#endif
+// One pair of softmax weights 2^(s*sl2 - m) on MUFU.EX2, after a scale-and-subtract
+// (packed float32x2 FMA when FP_PACKED_FMA is set, a compile-time tuning knob).
 #ifndef FP_PACKED_FMA
 #define FP_PACKED_FMA 1
 #endif
-constexpr int kEmuEvery = FP_EMU_EVERY;
-__device__ __forceinline__ bool emulated_pair(int pair) {
-  return kEmuEvery > 0 && (pair % (kEmuEvery > 0 ? kEmuEvery : 1)) == (kEmuEvery > 0 ? kEmuEvery : 1) - 1;
-}
 __device__ __forceinline__ void exp2_pair(float s0, float s1, float sl2, float m_ref, uint64_t sl2x2, uint64_t negm2,
-                                          bool emulate, float& p0, float& p1) {
-  if (emulate) {
-    exp2_poly2(f2_fma(f2_pack(s0, s1), sl2x2, negm2), p0, p1);
-  } else if (FP_PACKED_FMA) {
+                                          float& p0, float& p1) {
+  if (FP_PACKED_FMA) {
     float x0, x1;
     f2_unpack(f2_fma(f2_pack(s0, s1), sl2x2, negm2), x0, x1);
     p0 = fast_exp2(x0);
@@ -254,6 +211,7 @@ struct UnitIter {
   volatile int* abort;
   unsigned* status;
   bool producer;
+  bool warp;  // consumer called by whole warps (the softmax roles)
   long long num_units;
   long long u;
   int n;
@@ -277,7 +235,9 @@ struct UnitIter {
       mbar_arrive(full + slot);
       return v;
     }
-    if (!mbar_wait(full + slot, ph, abort, status, FP_DEV_TIMEOUT)) {
+    const bool got = warp ? mbar_wait<true>(full + slot, ph, abort, status, FP_DEV_TIMEOUT)
+                          : mbar_wait<false>(full + slot, ph, abort, status, FP_DEV_TIMEOUT);
+    if (!got) {
       ok = false;
       return LLONG_MAX;
     }
@@ -448,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       long long kt = 0, vt = 0, qn = 0;
       const uint32_t q_bytes = 2u * C::DCH * a.rows * 128u;
       bool ok = true;
-      UnitIter it{a.queue, a.order, unit_ring, unit_full, unit_empty, abort_flag, g.status, true, a.num_units, 0, 0};
+      UnitIter it{a.queue, a.order, unit_ring, unit_full, unit_empty, abort_flag, g.status, true, false, a.num_units, 0, 0};
       for (long long u = it.step(true, ok); u < a.num_units && ok; u = it.step(false, ok)) {
         Unit U;
         if (!decode_unit(u, a, U) || U.count == 0) continue;
@@ -479,15 +439,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++vt;
         }
       }
-      if (*abort_flag) {
-        // let every copy this CTA issued land before the shared memory is released
-        int never = 0;
-        for (long long t = kt - 1; t >= 0 && t >= kt - KS; --t)
-          mbar_wait(k_full + (int)(t % KS), (uint32_t)((t / KS) & 1), (volatile int*)&never, g.status, 0u);
-        for (long long t = vt - 1; t >= 0 && t >= vt - VS; --t)
-          mbar_wait(v_full + (int)(t % VS), (uint32_t)((t / VS) & 1), (volatile int*)&never, g.status, 0u);
-        if (qn > 0) mbar_wait(q_full, (uint32_t)((qn - 1) & 1), (volatile int*)&never, g.status, 0u);
-      }
+      // Every copy this CTA issued lands before its shared memory is released,
+      // also when another role gave up after this loop ended (on the normal
+      // path the consumers have already seen these phases complete).
+      for (long long t = kt - 1; t >= 0 && t >= kt - KS; --t)
+        mbar_drain(k_full + (int)(t % KS), (uint32_t)((t / KS) & 1), g.status, FP_DEV_TIMEOUT);
+      for (long long t = vt - 1; t >= 0 && t >= vt - VS; --t)
+        mbar_drain(v_full + (int)(t % VS), (uint32_t)((t / VS) & 1), g.status, FP_DEV_TIMEOUT);
+      if (qn > 0) mbar_drain(q_full, (uint32_t)((qn - 1) & 1), g.status, FP_DEV_TIMEOUT);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
@@ -536,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
 
-      UnitIter it{a.queue, a.order, unit_ring, unit_full, unit_empty, abort_flag, g.status, false, a.num_units, 0, 0};
+      UnitIter it{a.queue, a.order, unit_ring, unit_full, unit_empty, abort_flag, g.status, false, false, a.num_units, 0, 0};
       for (long long u = it.step(true, ok); u < a.num_units && ok; u = it.step(false, ok)) {
         Unit U;
         if (!decode_unit(u, a, U) || U.count == 0) continue;
@@ -605,8 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // every MMA this thread issued has completed once `drain` flips
       umma_commit(drain);
-      int never = 0;
-      mbar_wait(drain, 0u, (volatile int*)&never, g.status, FP_DEV_TIMEOUT);
+      mbar_drain(drain, 0u, g.status, FP_DEV_TIMEOUT);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax warpgroups
@@ -619,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int hh = row % g.G, tt = row / g.G;
     long long sn = 0, on = 0;
     bool ok = true;
-    UnitIter it{a.queue, a.order, unit_ring, unit_full, unit_empty, abort_flag, g.status, false, a.num_units, 0, 0};
+    UnitIter it{a.queue, a.order, unit_ring, unit_full, unit_empty, abort_flag, g.status, false, true, a.num_units, 0, 0};
     for (long long u = it.step(true, ok); u < a.num_units && ok; u = it.step(false, ok)) {
       Unit U;
       if (!decode_unit(u, a, U)) continue;
@@ -645,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int n = 0; n < U.count; ++n) {
         const uint32_t hb = hb_next;
         if (hbp && n + 1 < U.count) hb_next = __ldg(hbp + n + 1);  // one visit ahead
-        ok = mbar_wait(s_full + mt, (uint32_t)(sn & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
+        ok = mbar_wait<true>(s_full + mt, (uint32_t)(sn & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
         if (!ok) break;
         ++sn;
         tc_fence_after();
@@ -725,7 +683,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int e = 0; e < CH / 2; ++e) {
                 float p0, p1;
-                exp2_pair(s[k0 + 2 * e], s[k0 + 2 * e + 1], sl2, m_ref, sl2x2, negm2, emulated_pair(e), p0, p1);
+                exp2_pair(s[k0 + 2 * e], s[k0 + 2 * e + 1], sl2, m_ref, sl2x2, negm2, p0, p1);
                 const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
                 const uint32_t u = *reinterpret_cast<const uint32_t*>(&b2);
                 pk[e] = u;
@@ -753,8 +711,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int q = 0; q < 2; ++q) {
                 float x0, x1;
-                exp2_pair(s[32 * c + 4 * e + 2 * q], s[32 * c + 4 * e + 2 * q + 1], sl2, m_ref, sl2x2, negm2,
-                          emulated_pair(2 * e + q), x0, x1);
+                exp2_pair(s[32 * c + 4 * e + 2 * q], s[32 * c + 4 * e + 2 * q + 1], sl2, m_ref, sl2x2, negm2, x0,
+                          x1);
                 uint32_t h, r;
                 e4m3_split2(x0, x1, h, r);
                 if (q) {
@@ -791,7 +749,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         continue;
       }
-      ok = mbar_wait(o_full + mt, (uint32_t)(on & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
+      ok = mbar_wait<true>(o_full + mt, (uint32_t)(on & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
       if (!ok) break;
       ++on;
       tc_fence_after();

@@ -346,14 +346,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             for (int pl = 0; pl < 3; ++pl)
               tma_load_4d(sB + (st * 3 + pl) * kTile, &tmK, b_full + st, c * 64, nt * 128, rg, pl);
           }
-      if (*abort_flag) {
-        // let every copy this CTA issued land before the shared memory is released
-        int never = 0;
-        for (int t = n - 1; t >= 0 && t >= n - kScoreStages; --t)
-          mbar_wait(b_full + t % kScoreStages, (uint32_t)((t / kScoreStages) & 1), (volatile int*)&never,
-                    g.status, 0u);
-        mbar_wait(a_full, 0u, (volatile int*)&never, g.status, 0u);
-      }
+      // every copy this CTA issued lands before its shared memory is released,
+      // also when another role gave up after this loop ended
+      for (int t = n - 1; t >= 0 && t >= n - kScoreStages; --t)
+        mbar_drain(b_full + t % kScoreStages, (uint32_t)((t / kScoreStages) & 1), g.status, FP_DEV_TIMEOUT);
+      mbar_drain(a_full, 0u, g.status, FP_DEV_TIMEOUT);
     }
   } else if (warp == kScoreMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -389,8 +386,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
       // every MMA this thread issued has completed once `drain` flips
       umma_commit(drain);
-      int never = 0;
-      mbar_wait(drain, 0u, (volatile int*)&never, g.status, FP_DEV_TIMEOUT);
+      mbar_drain(drain, 0u, g.status, FP_DEV_TIMEOUT);
     }
   } else {
     // ------------------------------------------------------------ epilogue: thread = score row

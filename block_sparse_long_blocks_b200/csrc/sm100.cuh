@@ -24,8 +24,22 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Every pipeline wait gives up after this long (a healthy wait lasts microseconds).
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+// Every pipeline wait gives up after this long (a healthy wait lasts
+// microseconds). A build may lower it (-DFP_WAIT_LIMIT_NS=...) so that waits
+// run out on purpose and the abort path can be exercised.
+#ifndef FP_WAIT_LIMIT_NS
+#define FP_WAIT_LIMIT_NS 2000000000ull  // 2 s
+#endif
+constexpr uint64_t kWaitLimitNs = FP_WAIT_LIMIT_NS;
+// A short-limit build (under 1 ms) probes with the non-blocking test_wait and
+// reads the clock on every poll, so that any wait longer than the limit runs
+// out however long the hardware would let a try_wait suspend; otherwise the
+// clock is read every 64 polls of try_wait.
+constexpr bool kShortWaitBuild = kWaitLimitNs < 1000000ull;
+constexpr uint32_t kPollsPerClockRead = kShortWaitBuild ? 1u : 64u;
+// Drain waits (a CTA waiting for its own copies and MMAs before it releases
+// shared and tensor memory) always allow 2 s, whatever the pipeline limit.
+constexpr uint64_t kDrainLimitNs = 2000000000ull;
 
 // Per-warpgroup register limit changes (all four warps of the warpgroup execute them).
 template <uint32_t N>
@@ -70,23 +84,67 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
   return ok != 0;
 }
 
+// Non-blocking probe of the same condition.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar_addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase of `parity` to complete. Gives up after kWaitLimitNs or
 // as soon as *abort is set; on its own timeout it sets *abort and ORs `code`
 // into *status. Returns true when the phase completed.
+// WARP = true: called by all 32 lanes of a converged warp, which wait together
+// and all get the same answer (their callers go on to warp-collective tcgen05
+// instructions, so no lane may leave the wait alone).
+template <bool WARP = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           unsigned* status, unsigned code) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
+  auto done = [&]() -> bool {
+    const bool d = kShortWaitBuild ? mbar_test_wait(a, parity) : mbar_try_wait(a, parity);
+    if constexpr (WARP) return __all_sync(0xffffffffu, d) != 0;
+    return d;
+  };
+  if (done()) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(a, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        *abort = 1;
-        atomicOr(status, code);
-        return false;
+    if (done()) return true;
+    if (it % kPollsPerClockRead == 0) {
+      int stop = 0;
+      if (!WARP || (threadIdx.x & 31) == 0) {
+        if (*abort) {
+          stop = 1;
+        } else if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          *abort = 1;
+          atomicOr(status, code);
+          stop = 1;
+        }
       }
+      if constexpr (WARP) stop = __shfl_sync(0xffffffffu, stop, 0);
+      if (stop) return false;
+    }
+  }
+}
+
+// Waits (single thread, no abort flag) for a phase that the CTA's own
+// asynchronous work completes: a TMA copy landing or an MMA commit. Gives up
+// only after kDrainLimitNs, then ORs `code` into *status.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, unsigned* status, unsigned code) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(a, parity)) return;
+    if ((it & 63u) == 0 && globaltimer_ns() - t0 > kDrainLimitNs) {
+      atomicOr(status, code);
+      return;
     }
   }
 }

@@ -122,3 +122,13 @@ def test_alignment_workspace_and_pointer_checks(lib):
 def test_status_strings(lib):
     for code, name in fb.STATUS.items():
         assert lib.fp_status_string(code).decode() == name
+
+
+def test_short_wait_variant_builds_and_exports_the_same_symbols():
+    """The test build with a 500 ns pipeline-wait limit (abort-path test) is the
+    same library: same sources, same entry points."""
+    path = build.build_variant("short_wait")
+    short = fb.load_library(path)
+    for n in declared_functions():
+        assert hasattr(short, n), n
+    assert short.fp_static_scratch_bytes() == fb.load().fp_static_scratch_bytes()
