@@ -178,7 +178,8 @@ def test_full_path_tiny(fp8):
 
 
 def test_values_ones_and_zero_queries():
-    """V = 1 gives O = 1; Q = 0 gives the mean of V over the allowed keys (alpha = 0)."""
+    """V = 1 gives O = 1; Q = 0 gives, for every head and every channel, the mean
+    of the group's V over the keys up to the query (alpha = 0)."""
     w = _case("qwen30b_128k", 1000)
     inp = _inputs(w)
     inp.v = torch.ones_like(inp.v)
@@ -192,10 +193,16 @@ def test_values_ones_and_zero_queries():
     dev2 = H.Device(w, inp2, 0.0)
     dev2.discover()
     dev2.attend()
-    v = inp2.v[0, :, 0].double()
-    ref = torch.cumsum(v, 0) / torch.arange(1, v.shape[0] + 1, dtype=torch.float64)[:, None]
-    got = dev2.bufs.o[0, :, 0].double().cpu()
-    assert (got - ref).abs().max().item() <= 2e-2
+    n = torch.arange(1, inp2.v.shape[1] + 1, dtype=torch.float64)[:, None]
+    got = dev2.bufs.o[0].double().cpu()
+    worst = 0.0
+    for g in range(w.hkv):
+        ref = torch.cumsum(inp2.v[0, :, g].double(), 0) / n  # [L, d]
+        for h in range(g * w.group, (g + 1) * w.group):
+            e = (got[:, h] - ref).abs()
+            worst = max(worst, e.max().item())
+            assert e.max().item() <= 2e-2 and e.mean().item() <= 2e-3, (h, e.max().item())
+    print("Q = 0 closed form, all heads: max abs", worst)
 
 
 def test_empty_rows_give_zero_output():
@@ -297,35 +304,6 @@ def test_bad_cu_seqlens_reported():
     assert dev.status() & 2  # FP_DEV_BAD_SEQLENS
 
 
-# ----------------------------------------------------------------------------- full sizes (sampled)
-def _sample_rows(orc, w, r=0, k=6, seed=0):
-    N = orc[r]["mask"].shape[1]
-    dens = orc[r]["cnt"].sum(axis=0)
-    rng = np.random.default_rng(seed)
-    picks = {0, N - 1, N // 2, int(np.argmax(dens))} | set(rng.integers(0, N, k).tolist())
-    g_pick = rng.integers(0, w.hkv, len(picks)).tolist()
-    return {(r, g, i) for g, i in zip(g_pick, sorted(picks))}
-
-
-@pytest.mark.parametrize("fp8", [False, True])
-def test_full_size_128k(fp8):
-    w = W["qwen30b_128k"]
-    inp = _inputs(w, fp8)
-    dev = H.Device(w, inp)
-    dev.discover()
-    assert dev.status() == 0
-    orc = H.oracle_discovery(w, inp)
-    rep = {}
-    H.compare_lists(orc, dev.lists(), rep)
-    print("128K borderline blocks:", rep)
-    idx, cnt = H.upload_lists(dev.cfg, [o["lists"] for o in orc])
-    dev.attend(idx, cnt)
-    assert dev.status() == 0
-    rows = _sample_rows(orc, w)
-    H.check_attention(dev, H.oracle_attention(w, inp, orc, rows), fp8, rep)
-    print("128K attention:", rep)
-
-
 # ----------------------------------------------------------------------------- chunked prefill
 def _chunk_oracle(w, inp):
     """Oracle result per request of a chunked input (float64 of the exact inputs)."""
@@ -337,6 +315,45 @@ def _chunk_oracle(w, inp):
         V = H.f64(v, inp.v_scale)
         res.append((oracle.flashprefill_chunk(Qc, K, V, w.block, w.alpha, w.sink_tokens, w.window_tokens), row0))
     return res
+
+
+def _check_chunk_lists(dev, w, orc):
+    """GPU lists of a chunked input equal the oracle's up to borderline blocks;
+    returns the number of rows with a borderline difference."""
+    gl = dev.lists()
+    border = 0
+    for r, (o, _) in enumerate(orc):
+        N = o["mask"].shape[1]
+        for g in range(w.hkv):
+            for i in range(dev.cfg.nmax):
+                want = o["lists"][g][i].tolist() if i < N else []
+                if gl[r][g][i] != want:
+                    qb = np.stack([x if x is not None else np.zeros_like(o["kbar"][0, :1].repeat(w.hq, 0))
+                                   for x in o["qbar"]])
+                    b = oracle.row_borderline(qb, o["kbar"], o["scale"], w.alpha, g, i, H.BORDER_REL)
+                    assert set(gl[r][g][i]) ^ set(want) <= b, (r, g, i)
+                    border += 1
+    return border
+
+
+def _check_chunk_attention(dev, orc, fp8, label):
+    O = dev.bufs.o.double().cpu().numpy()
+    L = dev.bufs.lse.double().cpu().numpy()
+    errs, tot, n, lse_err = [], 0.0, 0, 0.0
+    for o, row0 in orc:
+        q_len = o["O"].shape[0]
+        e = np.abs(O[row0: row0 + q_len] - o["O"])
+        errs.append(e.max())
+        tot += e.sum()
+        n += e.size
+        lse_err = max(lse_err, float(np.abs(L[:, row0: row0 + q_len] - o["lse"]).max()))
+    mx, mean = max(errs), tot / n
+    print(label, "fp8" if fp8 else "bf16", dict(max_abs=mx, mean_abs=mean, lse=lse_err))
+    if fp8:
+        assert mx <= H.FP8_MAX
+    else:
+        assert mx <= H.BF16_MAX and mean <= H.BF16_MEAN
+    assert lse_err <= (2e-3 if fp8 else 5e-3)
 
 
 @pytest.mark.parametrize("fp8", [False, True])
@@ -351,38 +368,11 @@ def test_chunked_prefill_matches_oracle(fp8):
     dev.discover()
     assert dev.status() == 0
     orc = _chunk_oracle(w, inp)
-    gl = dev.lists()
-    border = 0
-    for r, (o, _) in enumerate(orc):
-        N = o["mask"].shape[1]
-        for g in range(w.hkv):
-            for i in range(dev.cfg.nmax):
-                want = o["lists"][g][i].tolist() if i < N else []
-                if gl[r][g][i] != want:
-                    qb = np.stack([x if x is not None else np.zeros_like(o["kbar"][0, :1].repeat(w.hq, 0))
-                                   for x in o["qbar"]])
-                    b = oracle.row_borderline(qb, o["kbar"], o["scale"], w.alpha, g, i, H.BORDER_REL)
-                    assert set(gl[r][g][i]) ^ set(want) <= b, (r, g, i)
-                    border += 1
+    border = _check_chunk_lists(dev, w, orc)
+    print("chunked borderline rows:", border)
     dev.attend()
     assert dev.status() == 0
-    O = dev.bufs.o.double().cpu().numpy()
-    L = dev.bufs.lse.double().cpu().numpy()
-    errs, tot, n, lse_err = [], 0.0, 0, 0.0
-    for o, row0 in orc:
-        q_len = o["O"].shape[0]
-        e = np.abs(O[row0: row0 + q_len] - o["O"])
-        errs.append(e.max())
-        tot += e.sum()
-        n += e.size
-        lse_err = max(lse_err, float(np.abs(L[:, row0: row0 + q_len] - o["lse"]).max()))
-    mx, mean = max(errs), tot / n
-    print("chunked", "fp8" if fp8 else "bf16", dict(max_abs=mx, mean_abs=mean, lse=lse_err, borderline_rows=border))
-    if fp8:
-        assert mx <= H.FP8_MAX
-    else:
-        assert mx <= H.BF16_MAX and mean <= H.BF16_MEAN
-    assert lse_err <= (2e-3 if fp8 else 5e-3)
+    _check_chunk_attention(dev, orc, fp8, "chunked")
 
 
 def test_block_aligned_chunk_equals_full_prefill_on_gpu():
@@ -548,3 +538,67 @@ def test_prefill_single_call_equals_separate_calls(case):
         assert torch.equal(a.head_bits, b.head_bits)
     assert torch.equal(a.bufs.o, b.bufs.o)
     assert torch.equal(torch.nan_to_num(a.bufs.lse, nan=7.0), torch.nan_to_num(b.bufs.lse, nan=7.0))
+
+
+def _run_prefill(w, inp, per_head):
+    from block_sparse_long_blocks_b200 import binding as fb
+    d = H.Device(w, inp, per_head=per_head)
+    d.bufs.o.zero_()
+    d.bufs.lse.fill_(float("nan"))
+    fb.fp_prefill(d.p, d.q, d.k, d.v, d.bufs.mask, d.bufs.idx, d.bufs.cnt, d.bufs.o, d.bufs.workspace, d.bufs.lse)
+    torch.cuda.synchronize()
+    assert d.status() == 0
+    return d
+
+
+def _keep_from_gpu(dev, w):
+    """Per-head selection [Hq, N, N] that the GPU's lists and head bits encode
+    (request 0), for the oracle's per-head attention."""
+    gl = dev.lists()[0]
+    bits = dev.head_bits.cpu().numpy()
+    N = dev.cfg.nmax
+    tri = N * (N + 1) // 2
+    keep = np.zeros((w.hq, N, N), dtype=bool)
+    for g in range(w.hkv):
+        for i in range(N):
+            base = g * tri + i * (i + 1) // 2
+            for n, j in enumerate(gl[g][i]):
+                for hh in range(w.group):
+                    keep[g * w.group + hh, i, j] = bool((bits[base + n] >> hh) & 1)
+    return keep
+
+
+@pytest.mark.parametrize("case", ["contig", "fp8", "paged", "chunked", "per_head"])
+def test_prefill_single_call_matches_oracle(case):
+    """fp_prefill (discovery, compaction, claim-order sort and attention in one
+    call) against the float64 oracle: lists bit-exact up to borderline blocks,
+    outputs within the bars. The oracle's attention runs on the lists the GPU
+    chose (each already checked against the oracle's own), so a borderline
+    block decided the other way cannot fail the output check."""
+    w, inp, per_head = _prefill_case(case)
+    fp8 = inp.dtype == "e4m3"
+    d = _run_prefill(w, inp, per_head)
+    if case == "chunked":
+        orc = _chunk_oracle(w, inp)
+        assert _check_chunk_lists(d, w, orc) == 0  # no borderline rows in this case: same lists
+        _check_chunk_attention(d, orc, fp8, "fp_prefill chunked")
+        return
+    orc = H.oracle_discovery(w, inp)
+    rep = {}
+    H.compare_lists(orc, d.lists(), rep)
+    gl = d.lists()
+    for r, o in enumerate(orc):
+        o["lists"] = [[np.asarray(gl[r][g][i], dtype=np.int64) for i in range(len(o["lists"][g]))]
+                      for g in range(w.hkv)]
+    if per_head:
+        _check_head_bits(d, w, H.oracle_discovery(w, inp))
+        q, k, v = H.request_views(inp)[0]
+        O, lse = oracle.per_head_attention(H.f64(q, inp.q_scale), H.f64(k, inp.k_scale), H.f64(v, inp.v_scale),
+                                           _keep_from_gpu(d, w), w.block, oracle.default_scale(w.head_dim))
+        e = np.abs(d.bufs.o[0].double().cpu().numpy() - O)
+        le = np.abs(d.bufs.lse.double().cpu().numpy() - lse).max()
+        print("fp_prefill per-head", dict(max_abs=e.max(), mean_abs=e.mean(), lse=le, **rep))
+        assert e.max() <= H.BF16_MAX and e.mean() <= H.BF16_MEAN and le <= 5e-3
+        return
+    H.check_attention(d, H.oracle_attention(w, inp, orc), fp8, rep)
+    print("fp_prefill", case, rep)
