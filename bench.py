@@ -71,16 +71,92 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
+FP8_PEAK_PATH = os.path.join(ROOT, "profiles", "fp8_peak.json")
+
+
 def peaks():
+    """Roofline denominators: HBM copy bandwidth and dense bf16 tensor throughput
+    from MEASURED_PEAKS.json; dense e4m3 (and f16) tensor throughput from
+    profiles/fp8_peak.json (measured by ``--measure-peaks``), else None."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
-                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
-                    fp8=float(d["fp8_tflops"]) if "fp8_tflops" in d else None, source="measured")
+        out = dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                   bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), source="measured")
     except (OSError, KeyError, ValueError):
-        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, fp8=None, source="fallback")
+        out = dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+    out["fp8"] = out["f16"] = None
+    try:
+        with open(FP8_PEAK_PATH) as f:
+            d = json.load(f)
+        out["fp8"] = float(d["e4m3_tflops"])
+        out["f16"] = float(d["f16_tflops"])
+    except (OSError, KeyError, ValueError):
+        pass
+    return out
+
+
+def measure_peaks(seconds: float = 4.0):
+    """Dense tensor-core throughput on this GPU, measured like the bf16 figure of
+    MEASURED_PEAKS.json: an 8192^3 product, best of 10 (CUDA events), for e4m3
+    (torch._scaled_mm, bf16 output, unit scales) and f16 (torch.matmul); the e4m3
+    one also back to back for a few seconds (sustained). Writes profiles/fp8_peak.json."""
+    n = 8192
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev).manual_seed(0)
+    a16 = torch.randn(n, n, device=dev, generator=g, dtype=torch.float16)
+    b16 = torch.randn(n, n, device=dev, generator=g, dtype=torch.float16)
+    a8 = a16.to(torch.float8_e4m3fn)
+    b8 = b16.to(torch.float8_e4m3fn).t().contiguous().t()  # column-major second operand
+    one = torch.ones((), device=dev, dtype=torch.float32)
+    fp8 = lambda: torch._scaled_mm(a8, b8, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)  # noqa: E731
+    f16 = lambda: torch.matmul(a16, b16)  # noqa: E731
+
+    def best(fn, reps=10):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return 2.0 * n ** 3 / (min(ts) * 1e-3) / 1e12
+
+    def sustained(fn):
+        clocks = ClockSampler(torch.cuda.current_device())
+        clocks.start()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        k, t0 = 0, time.time()
+        e0.record()
+        while time.time() - t0 < seconds:
+            for _ in range(20):
+                fn()
+            k += 20
+            torch.cuda.synchronize()
+        e1.record()
+        torch.cuda.synchronize()
+        clk = clocks.stop()
+        return 2.0 * n ** 3 * k / (e0.elapsed_time(e1) * 1e-3) / 1e12, clk
+
+    fp8_best, f16_best = best(fp8), best(f16)
+    fp8_sus, clk = sustained(fp8)
+    rec = {"e4m3_tflops": fp8_best, "e4m3_tflops_sustained": fp8_sus, "f16_tflops": f16_best,
+           "gpu_name": torch.cuda.get_device_name(), "torch": torch.__version__,
+           "when": time.strftime("%Y-%m-%dT%H:%M:%SZ", time.gmtime()),
+           "how": "8192^3 products (2*N^3 flops): torch._scaled_mm e4m3 x e4m3 -> bf16 with unit scales and "
+                  "torch.matmul f16, best of 10 with CUDA events; e4m3 also back to back for a few seconds "
+                  "(sustained)",
+           "clocks_sustained": clk}
+    os.makedirs(os.path.dirname(FP8_PEAK_PATH), exist_ok=True)
+    with open(FP8_PEAK_PATH, "w") as f:
+        json.dump(rec, f, indent=1)
+        f.write("\n")
+    print(json.dumps(rec), flush=True)
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -231,17 +307,25 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="qwen30b_128k")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "e4m3"])
+    ap.add_argument("--path", default="fused", choices=["fused", "unfused", "single"],
+                    help="fused: fp_discover_compact + attention (default); unfused: fp_discover + fp_compact + "
+                         "attention; single: fp_prefill (one call, device work queue)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-fp8-extra", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the 256K / paged / chunked measurements")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--measure-peaks", action="store_true",
+                    help="measure the dense e4m3 / f16 tensor-core peaks and write profiles/fp8_peak.json")
     ap.add_argument("--seq-len", type=int, default=0,
                     help="run a shorter sequence of the same workload (profiling small cases)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
 
+    if args.measure_peaks:
+        measure_peaks()
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -280,26 +364,33 @@ def run_reference(args, w, world):
     from tests import _helpers as H
     orc = H.oracle_discovery(w, inp)
     total_visits = int(sum(int(o["cnt"].sum()) for o in orc))
-    times = []
+    times, walls = [], []
     per_step_budget = max(2.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
     last = None
     for s in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
         smp = oracle_sample(w, inp, per_step_budget, max_rows=64, seed=s)
         if s >= args.warmup:
+            walls.append(time.perf_counter() - t0)
             times.append(extrapolate(smp, w, total_visits))
         last = smp
     t = statistics.mean(times)
     flops = w.dense_equiv_flops()
     val = flops / t / 1e12
+    # ms_per_step is what each step took on this machine's clock: a bounded
+    # sample of the layer; the whole layer's time is extrapolated from it.
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(walls) * 1e3,
+            "extrapolated_ms_per_layer": t * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "seq_len": w.seqlens[0], "hq": w.hq, "hkv": w.hkv, "block": w.block,
                        "alpha": w.alpha, "input_dtype": args.dtype},
             "cpu_baseline": {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                              "sample": f"per step {last['rows']} (KV group, query block) rows of the layer "
-                                       f"(discovery + attention) plus full key pooling, extrapolated by work "
-                                       f"counts to all {last['N'] * w.hkv} rows / {total_visits} visited blocks"},
+                                       f"(discovery + attention) plus full key pooling, timed "
+                                       f"({statistics.mean(walls):.1f} s per step) and extrapolated by work "
+                                       f"counts to all {last['N'] * w.hkv} rows / {total_visits} visited blocks "
+                                       f"(value = dense-equivalent flops / extrapolated_ms_per_layer)"},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -336,7 +427,18 @@ def run_native(args, w, world, rank, local, dist):
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        fb.fp_discover_compact(D["p"], D["q"], D["k"], None, D["bufs"].idx, D["bufs"].cnt, D["bufs"].workspace)
+        if args.path == "single":  # one call: discovery, claim-order sort, attention (no split)
+            fb.fp_prefill(D["p"], D["q"], D["k"], D["v"], None, D["bufs"].idx, D["bufs"].cnt, D["bufs"].o,
+                          D["bufs"].workspace)
+            if ev is not None:
+                ev[1].record(stream)
+                ev[2].record(stream)
+            return
+        if args.path == "unfused":
+            fb.fp_discover(D["p"], D["q"], D["k"], D["bufs"].mask, D["bufs"].workspace)
+            fb.fp_compact(D["p"], D["bufs"].mask, D["bufs"].idx, D["bufs"].cnt)
+        else:
+            fb.fp_discover_compact(D["p"], D["q"], D["k"], None, D["bufs"].idx, D["bufs"].cnt, D["bufs"].workspace)
         if ev is not None:
             ev[1].record(stream)
         if D["paged"]:
@@ -372,6 +474,8 @@ def run_native(args, w, world, rank, local, dist):
     ms = start.elapsed_time(end)
     disc_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    if args.path == "single":  # no event between the kernels of one call: the step is the attention's bound
+        disc_ms, attn_ms = float("nan"), statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     ms, disc_ms, attn_ms = max_over_ranks([ms, disc_ms, attn_ms], dist, dev)
     ms_step = ms / args.steps
 
@@ -398,7 +502,7 @@ def run_native(args, w, world, rank, local, dist):
                        "global_batch": world * len(w.seqlens), "hq": w.hq, "hkv": w.hkv, "head_dim": d,
                        "block": B, "alpha": w.alpha, "sink_tokens": w.sink_tokens,
                        "window_tokens": w.window_tokens, "parallelism": f"replicas{world} (one layer per rank)",
-                       "l2": "inputs larger than L2 (Q alone 1 GiB); no flush",
+                       "l2": "inputs larger than L2 (Q alone 1 GiB); no flush", "call_path": args.path,
                        "density": visits / causal_pairs},
             "ms_per_layer": ms_step, "discover_compact_ms": disc_ms, "attention_ms": attn_ms,
             "visited_tile_tflops": achieved,
@@ -411,9 +515,12 @@ def run_native(args, w, world, rank, local, dist):
                                    "peak": pk["hbm"], "unit": "GB/s",
                                    "frac": disc_bytes / (disc_ms * 1e-3) / 1e9 / pk["hbm"],
                                    "algorithmic_bytes": disc_bytes},
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": (3 if args.path == "fused" else 4) * args.steps,
             "clocks": clk}
 
+    if args.path == "single":
+        line["discover_compact_ms"] = None
+        line["discovery_roofline"] = None
     # end to end through the C ABI with host buffers (pinned), copies inside the timed region
     if not args.no_e2e:
         line["e2e"] = e2e(args, D, inp_host, dev, stream, dense, world, dist)
@@ -592,6 +699,41 @@ def e2e(args, D, inp_host, dev, stream, dense, world, dist):
     one(0)
     one(1)
     torch.cuda.synchronize()
+
+    # the parts on their own (device clocks), to show how much the pipeline overlaps
+    def timed_on(st, fn, reps=3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(st)
+        with torch.cuda.stream(st):
+            for _ in range(reps):
+                fn()
+        e1.record(st)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    b0 = sets[0]
+    h2d_ms = timed_on(s_in, lambda: (b0["q"].copy_(hq, non_blocking=True), b0["k"].copy_(hk, non_blocking=True),
+                                     b0["v"].copy_(hv, non_blocking=True)))
+    d2h_ms = timed_on(s_out, lambda: ho.copy_(b0["o"], non_blocking=True))
+    b1 = sets[1]
+    e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    torch.cuda.synchronize()
+    e0.record(s_in)
+    s_out.wait_event(e0)
+    with torch.cuda.stream(s_in):
+        for _ in range(3):
+            b1["q"].copy_(hq, non_blocking=True)
+            b1["k"].copy_(hk, non_blocking=True)
+            b1["v"].copy_(hv, non_blocking=True)
+    e1.record(s_in)
+    with torch.cuda.stream(s_out):
+        for _ in range(3):
+            ho.copy_(b0["o"], non_blocking=True)
+    e2.record(s_out)
+    torch.cuda.synchronize()
+    both_ms = max(e0.elapsed_time(e1), e0.elapsed_time(e2)) / 3
+    torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist is not None:
         dist.barrier()
@@ -603,7 +745,9 @@ def e2e(args, D, inp_host, dev, stream, dense, world, dist):
     ms = max_over_ranks([a.elapsed_time(b) / steps], dist, dev)[0]
     return {"value": weak_value(world, dense, ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps,
-            "pipelined": "two buffer sets, inputs / compute / output on three streams"}
+            "pipelined": "two buffer sets, inputs / compute / output on three streams",
+            "parts_ms": {"h2d_alone": h2d_ms, "d2h_alone": d2h_ms, "h2d_with_d2h_concurrent": both_ms,
+                         "h2d_GBps": h2d / (h2d_ms * 1e-3) / 1e9, "d2h_GBps": d2h / (d2h_ms * 1e-3) / 1e9}}
 
 
 def fp8_extra(args, w, inp_host, dev, stream, pk, setup, dist):
