@@ -17,12 +17,17 @@
 //   warp 8     TMA producer: Q tiles, then K[idx[n]] and V[idx[n]] into rings
 //   warp 9     MMA issuer (one thread): S = Q K^T into TMEM, O += P V with P
 //              read from TMEM (aliasing S), accumulators in TMEM
-//   warps 10-11 idle (complete the third warpgroup for the register split)
+//   warps 10-11 e4m3 inputs: widen each V tile to f16 in shared memory (exact)
+//              for the PV product; bf16 inputs: idle (they complete the third
+//              warpgroup for the register split)
+// Operand types: S = Q K^T on the input type (bf16, or e4m3 at twice the
+// tensor rate); P and V for O += P V are 16-bit (bf16, or f16 for e4m3
+// inputs: f16 keeps P to 2^-11 relative, where an e4m3 P would lose 2^-4).
 // Order of MMAs per visit n (ping-pong): PV0(n), S0(n+1), PV1(n), S1(n+1), so
 // one warpgroup's softmax overlaps the other tile's MMAs.
 // Softmax: online, base-2, with the running reference max raised only when the
-// tile max exceeds it by more than a threshold (64 for bf16, 8 for e4m3; then O
-// and l are rescaled in place).
+// tile max exceeds it by more than a threshold (64 for bf16 P, 15 for f16 P;
+// then O and l are rescaled in place).
 // Every wait is time-bounded; on expiry the CTA records FP_DEV_TIMEOUT, drains
 // its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -41,9 +46,14 @@ namespace {
 
 constexpr int kThreads = 384;  // 3 warpgroups
 constexpr int kUnitRing = 4;                // work units handed from the producer to the other roles
-constexpr int kUnitConsumers = 1 + 256;     // the MMA thread + both softmax warpgroups
+// the MMA thread + both softmax warpgroups (+ the two V-converter warps for e4m3)
+template <bool FP8>
+struct UnitConsumers {
+  static constexpr int value = 1 + 256 + (FP8 ? 64 : 0);
+};
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kConvertWarp = 10;  // warps 10-11 (e4m3 inputs)
 // Launched at 168 registers/thread (384 x 168 = 64512). The softmax warpgroups
 // then raise their limit and the producer/MMA warpgroup lowers its own:
 // 2 x 128 x 200 + 128 x 104 = 64512 <= 64512, and per SM sub-partition (three
@@ -54,30 +64,32 @@ constexpr uint32_t kControlRegs = 104;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * 168, "register split exceeds the launch");
 static_assert(2 * 32 * kSoftmaxRegs + 32 * kControlRegs <= 16384, "register split exceeds an SM sub-partition");
 // The reference max is raised only when a tile's max exceeds it by more than
-// this (log2 units); P is then at most 2^threshold. e4m3 P must stay below 448.
+// this (log2 units); P is then at most 2^threshold.
 // bf16 P, the float32 row sum and the float32 TMEM accumulators have float32's
 // exponent range: with 2^64 per weight, 2^18 keys and |v| < 2^4 every sum stays
 // below 2^86, so a rescale (a TMEM round trip of the O row) is needed only on
 // jumps of the row max by more than 64 (a factor 1.8e19).
+// f16 P (e4m3 inputs) must stay below 65504: threshold 15.
 #ifndef FP_RESCALE_LOG2_BF16
 #define FP_RESCALE_LOG2_BF16 64
 #endif
 template <bool FP8>
 struct RescaleThreshold {
-  static constexpr float value = FP8 ? 8.0f : (float)FP_RESCALE_LOG2_BF16;
+  static constexpr float value = FP8 ? 15.0f : (float)FP_RESCALE_LOG2_BF16;
 };
 // On a rescale the reference max is set this far below the new row max. For
-// e4m3 P this places the running max at P = 16 (P stays <= 2^8 = 256 < 448
-// because the threshold still bounds the reference gap at 8) and moves e4m3's
-// subnormal floor 16x further below it, so far fewer small weights underflow;
-// bf16 P has fp32's exponent range and needs no offset.
-#ifndef FP_E4M3_MAX_OFFSET
-#define FP_E4M3_MAX_OFFSET 4
+// f16 P this places the running max at P = 2^8 (P stays <= 2^15 because the
+// threshold still bounds the reference gap at 15) and moves f16's subnormal
+// floor (2^-24) a further 2^8 below it; bf16 P has float32's range and needs
+// no offset.
+#ifndef FP_F16P_MAX_OFFSET
+#define FP_F16P_MAX_OFFSET 8
 #endif
 template <bool FP8>
 struct MaxOffset {
-  static constexpr float value = FP8 ? (float)FP_E4M3_MAX_OFFSET : 0.0f;
+  static constexpr float value = FP8 ? (float)FP_F16P_MAX_OFFSET : 0.0f;
 };
+static_assert(FP_F16P_MAX_OFFSET <= 15, "f16 P would exceed 2^15");
 // Shared memory for the Q tiles and the K/V rings (the opt-in maximum per CTA is 227 KB).
 #ifndef FP_SMEM_BUDGET_KB
 #define FP_SMEM_BUDGET_KB 200
@@ -124,19 +136,46 @@ __device__ __forceinline__ void exp2_pair(float s0, float s1, float sl2, float m
   }
 }
 
-// e4m3 hi/lo planes of a pair (x0 low, x1 high), computed in f16x2: hi =
-// e4m3(x), lo = e4m3(x - hi). The f16 rounding of x (2^-11) is far below the
-// residual's own e4m3 rounding (2^-4 of |x - hi| <= 2^-8 |x|).
-__device__ __forceinline__ void e4m3_split2(float x0, float x1, uint32_t& hi16, uint32_t& lo16) {
-  unsigned short h8, l8;
-  uint32_t xh, hh, r;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(xh) : "f"(x1), "f"(x0));
-  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(h8) : "r"(xh));
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hh) : "h"(h8));
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(xh), "r"(hh));
-  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(l8) : "r"(r));
-  hi16 = h8;
-  lo16 = l8;
+// A pair of softmax weights as the PV product's 16-bit A operand (x0 in the
+// low half): f16 for e4m3 inputs, bf16 otherwise; round to nearest.
+template <bool F16>
+__device__ __forceinline__ uint32_t pack_p2(float x0, float x1) {
+  uint32_t u;
+  if constexpr (F16) {
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(x1), "f"(x0));
+  } else {
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(u) : "f"(x1), "f"(x0));
+  }
+  return u;
+}
+
+// e4m3 pair -> f16 pair (exact: every e4m3 value is an f16 value)
+__device__ __forceinline__ uint32_t widen_e4m3x2(uint32_t two_bytes) {
+  uint32_t u;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(u) : "h"((unsigned short)two_bytes));
+  return u;
+}
+
+// e4m3 V tile [BLK keys][128 d] as TMA wrote it (128-byte rows, 128-byte
+// swizzle: 16-byte granule p of row r sits at position p ^ (r & 7)) -> f16 tile
+// in the layout TMA gives a bf16 V tile: two chunks of 64 d-elements, each
+// [BLK keys][128 bytes] with the same swizzle. Thread ct of `nthreads` widens
+// granules ct, ct + nthreads, ...
+template <int BLK>
+__device__ __forceinline__ void widen_v_tile(const uint8_t* src, uint8_t* dst, int ct, int nthreads) {
+#pragma unroll 4
+  for (int q = ct; q < BLK * 8; q += nthreads) {
+    const int key = q >> 3, g8 = q & 7, sw = key & 7;
+    const uint4 w = *reinterpret_cast<const uint4*>(src + key * 128 + ((g8 ^ sw) << 4));
+    const uint4 lo = make_uint4(widen_e4m3x2(w.x), widen_e4m3x2(w.x >> 16), widen_e4m3x2(w.y),
+                                widen_e4m3x2(w.y >> 16));  // d = 16 g8 + 0..7
+    const uint4 hi = make_uint4(widen_e4m3x2(w.z), widen_e4m3x2(w.z >> 16), widen_e4m3x2(w.w),
+                                widen_e4m3x2(w.w >> 16));  // d = 16 g8 + 8..15
+    uint8_t* row = dst + (g8 >> 2) * (BLK * 128) + key * 128;
+    const int p = 2 * (g8 & 3);
+    *reinterpret_cast<uint4*>(row + ((p ^ sw) << 4)) = lo;
+    *reinterpret_cast<uint4*>(row + (((p + 1) ^ sw) << 4)) = hi;
+  }
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -145,12 +184,21 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// acc_lo += float(low bf16 of u); acc_hi += float(high bf16 of u)
-__device__ __forceinline__ void add_bf16x2(float& acc_lo, float& acc_hi, uint32_t u) {
-  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
-      : "+f"(acc_lo), "+f"(acc_hi)
-      : "r"(u));
+// acc_lo += float(low half of u); acc_hi += float(high half of u), u holding
+// two f16 (F16) or two bf16 values
+template <bool F16>
+__device__ __forceinline__ void add_p2(float& acc_lo, float& acc_hi, uint32_t u) {
+  if constexpr (F16) {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.f16 %0, lo, %0;\n\tadd.rn.f32.f16 %1, hi, %1;\n\t}"
+        : "+f"(acc_lo), "+f"(acc_hi)
+        : "r"(u));
+  } else {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+        : "+f"(acc_lo), "+f"(acc_hi)
+        : "r"(u));
+  }
 }
 
 struct AttnArgs {
@@ -171,29 +219,35 @@ struct AttnArgs {
 
 template <bool FP8, int BLK>
 struct Cfg {
-  static constexpr int ES = FP8 ? 1 : 2;
-  static constexpr int DCH = FP8 ? 1 : 2;                 // 128-byte chunks along d
+  static constexpr int ES = FP8 ? 1 : 2;                  // bytes per Q / K element
+  static constexpr int DCH = FP8 ? 1 : 2;                 // 128-byte chunks along d of Q, K (and loaded V)
   static constexpr int CH_ELEMS = 128 / DCH;              // elements per chunk
   static constexpr int Q_TILE = DCH * 128 * 128;          // bytes per 128-row M-tile
-  static constexpr int KV_CHUNK = BLK * 128;              // bytes per d-chunk of a K/V tile
-  static constexpr int KV_TILE = DCH * KV_CHUNK;
-  // K/V ring slots within the budget; an odd slot goes to K, whose tile is
-  // consumed about one visit before the V tile of the same block
-  static constexpr int TILES_RAW = (kSmemBudget - 2 * Q_TILE) / KV_TILE;
+  static constexpr int KV_CHUNK = BLK * 128;              // bytes per 128-byte-wide chunk of a K/V tile
+  static constexpr int K_TILE = DCH * KV_CHUNK;           // K tile (QK operand B)
+  static constexpr int V_TILE = 2 * KV_CHUNK;             // 16-bit V tile (PV operand B)
+  static constexpr int V8_TILE = FP8 ? KV_CHUNK : 0;      // e4m3 V tile as loaded
+  // Ring depths within the budget. bf16: K and V tiles have one size; an odd
+  // slot goes to K, whose tile is consumed about one visit before the V tile
+  // of the same block. e4m3: two f16 V slots, the rest shared by the e4m3 K
+  // and V rings.
+  static constexpr int REST = kSmemBudget - 2 * Q_TILE;
+  static constexpr int TILES_RAW = REST / K_TILE;
   static constexpr int TILES = TILES_RAW > 8 ? 8 : TILES_RAW;
-  static constexpr int V_STAGES = TILES / 2;
-  static constexpr int K_STAGES = TILES - V_STAGES;
-  static constexpr int KSTEP_BYTES = 32;                  // K extent of one MMA (16 bf16 / 32 e4m3)
-  static constexpr int QK_STEPS = 128 * ES / KSTEP_BYTES; // 8 (bf16) / 4 (e4m3)
-  static constexpr int PV_KEYS = KSTEP_BYTES / ES;        // keys per PV MMA: 16 / 32
+  static constexpr int N8 = FP8 ? (REST - 2 * V_TILE) / K_TILE : 0;
+  static constexpr int V_STAGES = FP8 ? 2 : TILES / 2;
+  static constexpr int K_STAGES = FP8 ? ((N8 + 1) / 2 > 4 ? 4 : (N8 + 1) / 2) : TILES - V_STAGES;
+  static constexpr int V8_STAGES = FP8 ? (N8 / 2 > 4 ? 4 : N8 / 2) : 0;
+  static constexpr int QK_STEPS = 128 * ES / 32;          // K = 32 bytes per MMA: 8 (bf16) / 4 (e4m3)
+  static constexpr int PV_KEYS = 16;                      // keys per 16-bit PV MMA
   static constexpr int PV_STEPS = BLK / PV_KEYS;
-  static constexpr int NUM_BARS = 2 + 2 * (K_STAGES + V_STAGES) + 8 + 1 + 2 * kUnitRing;
-  static constexpr int SMEM_USED =
-      1024 + 2 * Q_TILE + (K_STAGES + V_STAGES) * KV_TILE + NUM_BARS * 8 + 16 + 4 * kUnitRing;
+  static constexpr int NUM_BARS = 2 + 2 * (K_STAGES + V_STAGES + V8_STAGES) + 8 + 1 + 2 * kUnitRing;
+  static constexpr int SMEM_USED = 1024 + 2 * Q_TILE + K_STAGES * K_TILE + V_STAGES * V_TILE +
+                                   V8_STAGES * V8_TILE + NUM_BARS * 8 + 16 + 4 * kUnitRing;
   // more than half of the SM's shared memory: one CTA per SM, so the CTA's
   // 512-column TMEM allocation never waits for a co-resident CTA
   static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
-  static_assert(V_STAGES >= 2, "shared memory budget too small");
+  static_assert(V_STAGES >= 2 && K_STAGES >= 2 && (!FP8 || V8_STAGES >= 2), "shared memory budget too small");
   static_assert(SMEM <= 227 * 1024, "beyond the per-CTA shared memory limit");
 };
 
@@ -283,8 +337,17 @@ __device__ __forceinline__ bool decode_unit(long long u, const AttnArgs& a, Unit
   return true;
 }
 
-__device__ __forceinline__ int list_entry(const AttnArgs& a, const Unit& U, int n) {
-  int j = __ldg(a.idx + U.lbase + n);
+
+// The producer's view of one visited key block: its index and, for a paged
+// cache, the pool page of each page-sized sub-tile (at most BLK / 16 of them).
+// Loaded one visit ahead (raw), checked when the visit's copies are issued.
+template <int BLK>
+struct TileSrc {
+  int j;
+  int page[BLK / 16];
+};
+
+__device__ __forceinline__ int checked_entry(const AttnArgs& a, const Unit& U, int j) {
   if (j < 0 || j > U.i) {
     atomicOr(a.g.status, FP_DEV_BAD_LIST);
     j = U.i;
@@ -292,25 +355,42 @@ __device__ __forceinline__ int list_entry(const AttnArgs& a, const Unit& U, int 
   return j;
 }
 
+// Raw page-table entries of the sub-tiles of block j (paged only).
+template <int BLK>
+__device__ __forceinline__ void load_pages(const AttnArgs& a, const Unit& U, TileSrc<BLK>& t) {
+  const Geometry& g = a.g;
+  const int sub_rows = g.page_size < BLK ? g.page_size : BLK;
+  const int nsub = BLK / sub_rows;
+  const int32_t* row = g.page_table + (long long)U.r * g.max_pages;
+#pragma unroll
+  for (int s = 0; s < BLK / 16; ++s) {
+    const int tok = t.j * BLK + s * sub_rows;
+    t.page[s] = (s < nsub && tok < U.len) ? __ldg(row + (tok >> g.page_shift)) : g.num_pages;
+  }
+}
+
+// Copies of the K or V tile of a visited block whose pages were loaded raw:
+// out-of-range page ids are reported and read as zeros (outside the pool).
 template <bool FP8, int BLK, bool PAGED>
-__device__ __forceinline__ void load_kv_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
-                                             const AttnArgs& a, const Unit& U, int j) {
+__device__ __forceinline__ void issue_kv_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, const AttnArgs& a,
+                                              const Unit& U, const TileSrc<BLK>& t) {
   using C = Cfg<FP8, BLK>;
   const Geometry& g = a.g;
   if constexpr (!PAGED) {
 #pragma unroll
     for (int ch = 0; ch < C::DCH; ++ch)
-      tma_load_3d(dst + ch * C::KV_CHUNK, map, bar, ch * C::CH_ELEMS, U.kvh, U.off + j * BLK);
+      tma_load_3d(dst + ch * C::KV_CHUNK, map, bar, ch * C::CH_ELEMS, U.kvh, U.off + t.j * BLK);
   } else {
     const int sub_rows = g.page_size < BLK ? g.page_size : BLK;
     const int nsub = BLK / sub_rows;
-    for (int s = 0; s < nsub; ++s) {
-      const int tok = j * BLK + s * sub_rows;
-      int page = g.num_pages;  // out of range -> the copy fills zeros
-      if (tok < U.len) {
-        const int pg = __ldg(g.page_table + (long long)U.r * g.max_pages + (tok >> g.page_shift));
-        if (pg >= 0 && pg < g.num_pages) page = pg;
-        else atomicOr(g.status, FP_DEV_BAD_PAGE);
+#pragma unroll
+    for (int s = 0; s < BLK / 16; ++s) {
+      if (s >= nsub) break;
+      const int tok = t.j * BLK + s * sub_rows;
+      int page = t.page[s];
+      if (tok < U.len && (page < 0 || page >= g.num_pages)) {
+        atomicOr(g.status, FP_DEV_BAD_PAGE);
+        page = g.num_pages;  // out of range -> the copy fills zeros
       }
       const int slot = tok & (g.page_size - 1);
 #pragma unroll
@@ -325,20 +405,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     sparse_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   using C = Cfg<FP8, BLK>;
-  constexpr int KS = C::K_STAGES, VS = C::V_STAGES;
+  constexpr int KS = C::K_STAGES, VS = C::V_STAGES, V8S = C::V8_STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + 2 * C::Q_TILE;
-  uint8_t* sV = sK + KS * C::KV_TILE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VS * C::KV_TILE);
+  uint8_t* sV = sK + KS * C::K_TILE;    // 16-bit V tiles (PV operand)
+  uint8_t* sV8 = sV + VS * C::V_TILE;   // e4m3 V tiles as loaded (e4m3 inputs)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV8 + V8S * C::V8_TILE);
   uint64_t* q_full = bars;
   uint64_t* q_empty = bars + 1;
   uint64_t* k_full = bars + 2;
   uint64_t* k_empty = k_full + KS;
   uint64_t* v_full = k_empty + KS;
   uint64_t* v_empty = v_full + VS;
-  uint64_t* s_full = v_empty + VS;  // [2]
+  uint64_t* v8_full = v_empty + VS;   // [V8S]
+  uint64_t* v8_empty = v8_full + V8S;  // [V8S]
+  uint64_t* s_full = v8_empty + V8S;  // [2]
   uint64_t* p_full = s_full + 2;   // [M-tile][half of the keys]
   uint64_t* o_full = p_full + 4;   // [2]
   uint64_t* drain = o_full + 2;
@@ -359,8 +442,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(k_empty + s, 1);
     }
     for (int s = 0; s < VS; ++s) {
-      mbar_init(v_full + s, 1);
+      mbar_init(v_full + s, FP8 ? 64 : 1);  // e4m3: every converter thread arrives
       mbar_init(v_empty + s, 1);
+    }
+    for (int s = 0; s < V8S; ++s) {
+      mbar_init(v8_full + s, 1);
+      mbar_init(v8_empty + s, 64);
     }
     for (int m = 0; m < 2; ++m) {
       mbar_init(s_full + m, 1);
@@ -371,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(drain, 1);
     for (int k = 0; k < kUnitRing; ++k) {
       mbar_init(unit_full + k, 1);
-      mbar_init(unit_empty + k, kUnitConsumers);
+      mbar_init(unit_empty + k, UnitConsumers<FP8>::value);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -407,6 +494,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmV);
       long long kt = 0, vt = 0, qn = 0;
       const uint32_t q_bytes = 2u * C::DCH * a.rows * 128u;
+      constexpr int VLS = FP8 ? V8S : VS;
+      constexpr int VL_TILE = FP8 ? C::V8_TILE : C::V_TILE;
+      uint8_t* sVL = FP8 ? sV8 : sV;
+      uint64_t* vl_full = FP8 ? v8_full : v_full;
+      uint64_t* vl_empty = FP8 ? v8_empty : v_empty;
       bool ok = true;
       UnitIter it{a.queue, a.order, unit_ring, unit_full, unit_empty, abort_flag, g.status, true, false, a.num_units, 0, 0};
       for (long long u = it.step(true, ok); u < a.num_units && ok; u = it.step(false, ok)) {
@@ -423,20 +515,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(sQ + mt * C::Q_TILE + ch * 128 * 128, &tmQ, q_full, ch * C::CH_ELEMS, U.kvh * g.G, t);
         }
         ++qn;
+        // Tile sources run ahead of the copies: the list entry of visit n + 2
+        // and the pages of visit n + 1 are loaded before the producer blocks on
+        // the rings for visit n, so their latency hides behind those waits.
+        const int32_t* lrow = a.idx + U.lbase;
+        TileSrc<BLK> cur, nxt;
+        cur.j = checked_entry(a, U, __ldg(lrow));
+        if constexpr (PAGED) load_pages<BLK>(a, U, cur);
+        int j_ahead = U.count > 1 ? __ldg(lrow + 1) : 0;
         for (int n = 0; n < U.count && ok; ++n) {
-          const int j = list_entry(a, U, n);
+          if (n + 1 < U.count) {
+            nxt.j = checked_entry(a, U, j_ahead);
+            if constexpr (PAGED) load_pages<BLK>(a, U, nxt);
+            if (n + 2 < U.count) j_ahead = __ldg(lrow + n + 2);
+          }
           int st = (int)(kt % KS);
           ok = mbar_wait(k_empty + st, (uint32_t)((kt / KS) & 1) ^ 1u, abort_flag, g.status, FP_DEV_TIMEOUT);
           if (!ok) break;
-          mbar_arrive_expect_tx(k_full + st, C::KV_TILE);
-          load_kv_tile<FP8, BLK, PAGED>(sK + st * C::KV_TILE, &tmK, k_full + st, a, U, j);
+          mbar_arrive_expect_tx(k_full + st, C::K_TILE);
+          issue_kv_tile<FP8, BLK, PAGED>(sK + st * C::K_TILE, &tmK, k_full + st, a, U, cur);
           ++kt;
-          st = (int)(vt % VS);
-          ok = mbar_wait(v_empty + st, (uint32_t)((vt / VS) & 1) ^ 1u, abort_flag, g.status, FP_DEV_TIMEOUT);
+          // V: straight into the 16-bit ring (bf16) or into the e4m3 ring the converter reads
+          st = (int)(vt % VLS);
+          ok = mbar_wait(vl_empty + st, (uint32_t)((vt / VLS) & 1) ^ 1u, abort_flag, g.status, FP_DEV_TIMEOUT);
           if (!ok) break;
-          mbar_arrive_expect_tx(v_full + st, C::KV_TILE);
-          load_kv_tile<FP8, BLK, PAGED>(sV + st * C::KV_TILE, &tmV, v_full + st, a, U, j);
+          mbar_arrive_expect_tx(vl_full + st, VL_TILE);
+          issue_kv_tile<FP8, BLK, PAGED>(sVL + st * VL_TILE, &tmV, vl_full + st, a, U, cur);
           ++vt;
+          cur = nxt;
         }
       }
       // Every copy this CTA issued lands before its shared memory is released,
@@ -444,13 +550,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       // path the consumers have already seen these phases complete).
       for (long long t = kt - 1; t >= 0 && t >= kt - KS; --t)
         mbar_drain(k_full + (int)(t % KS), (uint32_t)((t / KS) & 1), g.status, FP_DEV_TIMEOUT);
-      for (long long t = vt - 1; t >= 0 && t >= vt - VS; --t)
-        mbar_drain(v_full + (int)(t % VS), (uint32_t)((t / VS) & 1), g.status, FP_DEV_TIMEOUT);
+      for (long long t = vt - 1; t >= 0 && t >= vt - VLS; --t)
+        mbar_drain(vl_full + (int)(t % VLS), (uint32_t)((t / VLS) & 1), g.status, FP_DEV_TIMEOUT);
       if (qn > 0) mbar_drain(q_full, (uint32_t)((qn - 1) & 1), g.status, FP_DEV_TIMEOUT);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      // QK: kind::f8f6f4 e4m3 (format 0) or kind::f16 bf16 (format 1);
+      // PV: kind::f16, f16 (format 0) for e4m3 inputs or bf16 (format 1)
       const uint32_t fmt = FP8 ? 0u : 1u;
       const uint32_t idesc_qk = instr_desc(fmt, 128, BLK, 0, 0);
       const uint32_t idesc_pv = instr_desc(fmt, 128, 128, 0, 1);
@@ -467,10 +575,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dV = smem_desc_sw128(sVa, C::KV_CHUNK, 1024);
       auto issue_qk = [&](int mt, int kst) {
         const uint64_t a0 = dQ + (uint64_t)((mt * C::Q_TILE) >> 4);
-        const uint64_t b0 = dK + (uint64_t)((kst * C::KV_TILE) >> 4);
+        const uint64_t b0 = dK + (uint64_t)((kst * C::K_TILE) >> 4);
 #pragma unroll
         for (int ks = 0; ks < C::QK_STEPS; ++ks) {
-          const uint32_t boff = (uint32_t)(ks * C::KSTEP_BYTES);
+          const uint32_t boff = (uint32_t)(ks * 32);  // 32 bytes of K per MMA
           const uint32_t ch = boff / 128, in = boff % 128;
           const uint64_t ad = a0 + ((ch * 128 * 128 + in) >> 4);
           const uint64_t bd = b0 + ((ch * C::KV_CHUNK + in) >> 4);
@@ -478,20 +586,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           else umma_f16_ss(tmem + mt * 128, ad, bd, idesc_qk, ks > 0);
         }
       };
-      // P occupies the first columns of the M-tile's S region: bf16 pairs, or for
-      // e4m3 a high plane (BLK/4 columns) followed by the residual plane.
+      // P occupies the first BLK / 2 columns of the M-tile's S region (16-bit pairs).
       auto issue_pv = [&](int mt, int vst, bool acc, int hf) {
-        const uint64_t b0 = dV + (uint64_t)((vst * C::KV_TILE) >> 4);
+        const uint64_t b0 = dV + (uint64_t)((vst * C::V_TILE) >> 4);
 #pragma unroll
-        for (int plane = 0; plane < (FP8 ? 2 : 1); ++plane) {
-#pragma unroll
-          for (int ks = hf * (C::PV_STEPS / 2); ks < (hf + 1) * (C::PV_STEPS / 2); ++ks) {
-            const uint32_t a_t = tmem + mt * 128 + plane * (BLK / 4) + ks * (C::PV_KEYS * C::ES / 4);
-            const uint64_t bd = b0 + ((ks * C::PV_KEYS * 128) >> 4);
-            const uint32_t accum = (acc || ks > 0 || plane > 0) ? 1u : 0u;
-            if (FP8) umma_f8_ts(tmem + 256 + mt * 128, a_t, bd, idesc_pv, accum);
-            else umma_f16_ts(tmem + 256 + mt * 128, a_t, bd, idesc_pv, accum);
-          }
+        for (int ks = hf * (C::PV_STEPS / 2); ks < (hf + 1) * (C::PV_STEPS / 2); ++ks) {
+          const uint32_t a_t = tmem + mt * 128 + ks * (C::PV_KEYS / 2);
+          const uint64_t bd = b0 + ((ks * C::PV_KEYS * 128) >> 4);
+          umma_f16_ts(tmem + 256 + mt * 128, a_t, bd, idesc_pv, (acc || ks > 0) ? 1u : 0u);
         }
       };
 
@@ -565,6 +667,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every MMA this thread issued has completed once `drain` flips
       umma_commit(drain);
       mbar_drain(drain, 0u, g.status, FP_DEV_TIMEOUT);
+    }
+  } else if (FP8 && warp >= kConvertWarp) {
+    // ------------------------------------------------------------------ V converter (e4m3 inputs)
+    // Widens every V tile the producer loads, in the same order, from the e4m3
+    // ring into the f16 ring the PV MMAs read; exact (e4m3 is a subset of f16).
+    const int ct = threadIdx.x - kConvertWarp * 32;  // 0..63
+    long long vt = 0;
+    bool ok = true;
+    UnitIter it{a.queue, a.order, unit_ring, unit_full, unit_empty, abort_flag, g.status, false, true, a.num_units, 0, 0};
+    for (long long u = it.step(true, ok); u < a.num_units && ok; u = it.step(false, ok)) {
+      Unit U;
+      if (!decode_unit(u, a, U) || U.count == 0) continue;
+      for (int n = 0; n < U.count; ++n, ++vt) {
+        constexpr int V8D = V8S > 0 ? V8S : 1;  // (this branch runs for e4m3 only)
+        const int s8 = (int)(vt % V8D), s16 = (int)(vt % VS);
+        ok = mbar_wait<true>(v8_full + s8, (uint32_t)((vt / V8D) & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
+        if (!ok) break;
+        ok = mbar_wait<true>(v_empty + s16, (uint32_t)((vt / VS) & 1) ^ 1u, abort_flag, g.status, FP_DEV_TIMEOUT);
+        if (!ok) break;
+        widen_v_tile<BLK>(sV8 + s8 * C::V8_TILE, sV + s16 * C::V_TILE, ct, 64);
+        // the tensor cores read the tile through the async proxy
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(v_full + s16);
+        mbar_arrive(v8_empty + s8);
+      }
+      if (!ok) break;
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax warpgroups
@@ -659,19 +787,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st16(tO + c * 16, r16);
           }
         }
-        // P = 2^(s*sl2 - m_ref), computed where it is packed.
-        // bf16: the row sum is taken over the rounded weights that the PV MMA
-        // consumes, so O / l is an exact convex combination of V rows and a
-        // dominant key's rounding cancels between numerator and denominator.
-        // e4m3: the row sum is over the float32 weights, which also accounts
-        // for the mass of weights below the e4m3 subnormal floor.
+        // P = 2^(s*sl2 - m_ref), computed where it is packed (bf16, or f16 for
+        // e4m3 inputs). The row sum is taken over the rounded weights that the
+        // PV MMA consumes, so O / l is an exact convex combination of V rows
+        // and a dominant key's rounding cancels between numerator and denominator.
         float lsum0 = 0.f, lsum1 = 0.f, lsum2 = 0.f, lsum3 = 0.f;
         // (m_ref stays -inf while every visited block so far was masked for this row)
         const float negm = m_ref == -INFINITY ? 0.f : -m_ref;
         const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(negm, negm);
         // P goes out in two halves of the visited block's keys; the MMA issuer
         // starts O += P V on the first half while the second is computed.
-        if constexpr (!FP8) {
+        {
           constexpr int HALF = BLK / 2;              // keys per half
           constexpr int CH = HALF < 64 ? HALF : 64;  // keys per TMEM store
 #pragma unroll
@@ -684,11 +810,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int e = 0; e < CH / 2; ++e) {
                 float p0, p1;
                 exp2_pair(s[k0 + 2 * e], s[k0 + 2 * e + 1], sl2, m_ref, sl2x2, negm2, p0, p1);
-                const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-                const uint32_t u = *reinterpret_cast<const uint32_t*>(&b2);
+                const uint32_t u = pack_p2<FP8>(p0, p1);
                 pk[e] = u;
-                if (e & 1) add_bf16x2(lsum2, lsum3, u);
-                else add_bf16x2(lsum0, lsum1, u);
+                if (e & 1) add_p2<FP8>(lsum2, lsum3, u);
+                else add_p2<FP8>(lsum0, lsum1, u);
               }
               if constexpr (CH == 64) tmem_st32(tS + k0 / 2, pk);
               else tmem_st16(tS + k0 / 2, pk);
@@ -696,45 +821,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(p_full + 2 * mt + hf);
-          }
-        } else {
-          // P = hi + lo, both e4m3: the residual plane keeps the weights' relative
-          // error near 2^-8 instead of e4m3's 2^-4. Planes: hi in columns
-          // [0, BLK/4), lo in [BLK/4, BLK/2); packed 32 values (8 columns) at a time.
-#pragma unroll
-          for (int c = 0; c < BLK / 32; ++c) {
-            const int hf = c / (BLK / 64);
-            uint32_t phi[8], plo[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              uint32_t h32 = 0, l32 = 0;
-#pragma unroll
-              for (int q = 0; q < 2; ++q) {
-                float x0, x1;
-                exp2_pair(s[32 * c + 4 * e + 2 * q], s[32 * c + 4 * e + 2 * q + 1], sl2, m_ref, sl2x2, negm2, x0,
-                          x1);
-                uint32_t h, r;
-                e4m3_split2(x0, x1, h, r);
-                if (q) {
-                  lsum2 += x0;
-                  lsum3 += x1;
-                } else {
-                  lsum0 += x0;
-                  lsum1 += x1;
-                }
-                h32 |= h << (16 * q);
-                l32 |= r << (16 * q);
-              }
-              phi[e] = h32;
-              plo[e] = l32;
-            }
-            tmem_st8(tS + 8 * c, phi);
-            tmem_st8(tS + BLK / 4 + 8 * c, plo);
-            if (c % (BLK / 64) == BLK / 64 - 1) {  // last chunk of a half
-              tmem_wait_st();
-              tc_fence_before();
-              mbar_arrive(p_full + 2 * mt + hf);
-            }
           }
         }
         l += (lsum0 + lsum1) + (lsum2 + lsum3);

@@ -172,9 +172,12 @@ fp_status_t fp_discover_compact(const fp_params_t* p, const void* q, const void*
  * q, k, v: contiguous or varlen layout (no page table; p->page_table must be
  * NULL). o: device bf16, same layout as q. lse: NULL or device float
  * [hq, R * max_seqlen] (contiguous) / [hq, total_tokens] (varlen), natural-log
- * sum of exponentials of the scaled logits. With bf16 inputs O is normalised
- * by the sum of the bf16-rounded softmax weights the PV product uses, and lse
- * is the log of that same sum (within 2^-8 relative of the exact sum). Rows
+ * sum of exponentials of the scaled logits. S = Q K^T runs on the input type
+ * (bf16, or e4m3 with float32 accumulation); the softmax weights P and V enter
+ * O += P V as 16-bit values: bf16 for bf16 inputs, f16 for e4m3 inputs (V is
+ * widened exactly from e4m3 to f16 on chip). O is normalised by the sum of the
+ * rounded weights the PV product uses, and lse is the log of that same sum
+ * (within 2^-8 relative of the exact sum for bf16, 2^-11 for f16). Rows
  * with cnt = 0 get O = 0 and lse = -inf. Output rows of tokens outside every
  * request are not written.
  */
