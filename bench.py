@@ -603,6 +603,20 @@ def extra_workloads(args, setup, stream, pk, fp8):
                 disc.append(ev[0].elapsed_time(ev[1]))
                 attn.append(ev[1].elapsed_time(ev[2]))
                 tot.append(ev[0].elapsed_time(ev[2]))
+        single = None
+        if name in ("paged_varlen", "chunked_prefill_last_quarter"):
+            # the same layer through fp_prefill: one call, longest lists claimed first
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            st = []
+            for s in range(3 + 5):
+                e0.record(stream)
+                fb.fp_prefill(D["p"], D["q"], D["k"], D["v"], None, D["bufs"].idx, D["bufs"].cnt, D["bufs"].o,
+                              D["bufs"].workspace)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                if s >= 3:
+                    st.append(e0.elapsed_time(e1))
+            single = statistics.mean(st)
         cnt = D["bufs"].cnt.long()
         visits = int(cnt.sum().item())
         flops = visits * 4.0 * w.block * w.block * w.head_dim * w.group
@@ -617,6 +631,8 @@ def extra_workloads(args, setup, stream, pk, fp8):
                      "dense_equiv_tflops": dense / (t * 1e-3) / 1e12,
                      "visited_tile_tflops": flops / (a * 1e-3) / 1e12, "frac_of_peak": flops / (a * 1e-3) / 1e12 / peak,
                      "visited_blocks": visits, "tokens": int(inp.q.shape[0] * (inp.q.shape[1] if inp.q.dim() == 4 else 1))}
+        if single is not None:
+            out[name]["single_call_ms_per_layer"] = single
         del D, inp
         torch.cuda.empty_cache()
     return out

@@ -144,13 +144,14 @@ def config_for(w, inp, alpha: Optional[float] = None) -> Config:
     fp8 = inp.dtype == "e4m3"
     if inp.cu_seqlens is None:
         return Config(batch=inp.q.shape[0], max_seqlen=inp.q.shape[1], hq=w.hq, hkv=w.hkv, block=w.block,
-                      alpha=a, sink_tokens=w.sink_tokens, window_tokens=w.window_tokens, fp8=fp8)
+                      alpha=a, sink_tokens=w.sink_tokens, window_tokens=w.window_tokens, fp8=fp8,
+                      head_dim=w.head_dim)
     lens = (inp.cu_seqlens[1:] - inp.cu_seqlens[:-1]).tolist()
     if getattr(inp, "kv_lens", None) is not None:
         lens = inp.kv_lens.tolist()
     paged = inp.page_table is not None
     return Config(batch=len(lens), max_seqlen=max(lens), hq=w.hq, hkv=w.hkv, block=w.block, alpha=a,
-                  sink_tokens=w.sink_tokens, window_tokens=w.window_tokens, fp8=fp8,
+                  sink_tokens=w.sink_tokens, window_tokens=w.window_tokens, fp8=fp8, head_dim=w.head_dim,
                   total_tokens=int(inp.cu_seqlens[-1]), page_size=w.page_size if paged else 0,
                   max_pages_per_req=inp.page_table.shape[1] if paged else 0,
                   num_pages=inp.k_pool.shape[0] if paged else 0)

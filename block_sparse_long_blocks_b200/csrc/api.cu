@@ -55,7 +55,9 @@ fp_status_t validate(const fp_params_t* p, bool attention) {
   if (!std::isfinite(p->alpha) || p->alpha < 0.f) return FP_ERR_INVALID_ARG;
   if (p->sink_tokens < 0 || p->window_tokens < 0) return FP_ERR_INVALID_ARG;
   if (!std::isfinite(p->softmax_scale) || p->softmax_scale < 0.f) return FP_ERR_INVALID_ARG;
-  if (p->head_dim != 128) return FP_ERR_UNSUPPORTED;
+  // head dim 128, or 64 with bf16 inputs (an e4m3 row of 64 would be 64 bytes,
+  // below the kernels' 128-byte swizzled rows)
+  if (p->head_dim != 128 && !(p->head_dim == 64 && p->dtype == FP_BF16)) return FP_ERR_UNSUPPORTED;
   if (p->block != 64 && p->block != 128) return FP_ERR_UNSUPPORTED;
   const int G = p->hq / p->hkv;
   if (!(G <= 8 || G == 16)) return FP_ERR_UNSUPPORTED;

@@ -217,16 +217,19 @@ struct AttnArgs {
   const int* order;    // with a queue: the units in claim order (longest lists first)
 };
 
-template <bool FP8, int BLK>
+template <bool FP8, int BLK, int D>
 struct Cfg {
   static constexpr int ES = FP8 ? 1 : 2;                  // bytes per Q / K element
-  static constexpr int DCH = FP8 ? 1 : 2;                 // 128-byte chunks along d of Q, K (and loaded V)
-  static constexpr int CH_ELEMS = 128 / DCH;              // elements per chunk
+  static constexpr int ROW = D * ES;                      // bytes of one Q / K row
+  static constexpr int DCH = ROW / 128;                   // 128-byte chunks along d of Q, K (and loaded V)
+  static constexpr int CH_ELEMS = 128 / ES;               // elements per chunk
   static constexpr int Q_TILE = DCH * 128 * 128;          // bytes per 128-row M-tile
   static constexpr int KV_CHUNK = BLK * 128;              // bytes per 128-byte-wide chunk of a K/V tile
   static constexpr int K_TILE = DCH * KV_CHUNK;           // K tile (QK operand B)
-  static constexpr int V_TILE = 2 * KV_CHUNK;             // 16-bit V tile (PV operand B)
-  static constexpr int V8_TILE = FP8 ? KV_CHUNK : 0;      // e4m3 V tile as loaded
+  static constexpr int V_TILE = (D / 64) * KV_CHUNK;      // 16-bit V tile (PV operand B, 64 d per chunk)
+  static constexpr int V8_TILE = FP8 ? DCH * KV_CHUNK : 0;  // e4m3 V tile as loaded
+  static_assert(ROW % 128 == 0 && (D == 64 || D == 128), "head dim 64 (16-bit inputs) or 128");
+  static_assert(!FP8 || D == 128, "e4m3 inputs need 128-byte rows: head dim 128");
   // Ring depths within the budget. bf16: K and V tiles have one size; an odd
   // slot goes to K, whose tile is consumed about one visit before the V tile
   // of the same block. e4m3: two f16 V slots, the rest shared by the e4m3 K
@@ -238,7 +241,7 @@ struct Cfg {
   static constexpr int V_STAGES = FP8 ? 2 : TILES / 2;
   static constexpr int K_STAGES = FP8 ? ((N8 + 1) / 2 > 4 ? 4 : (N8 + 1) / 2) : TILES - V_STAGES;
   static constexpr int V8_STAGES = FP8 ? (N8 / 2 > 4 ? 4 : N8 / 2) : 0;
-  static constexpr int QK_STEPS = 128 * ES / 32;          // K = 32 bytes per MMA: 8 (bf16) / 4 (e4m3)
+  static constexpr int QK_STEPS = ROW / 32;               // K = 32 bytes per MMA: 8 (bf16) / 4 (e4m3) at d = 128
   static constexpr int PV_KEYS = 16;                      // keys per 16-bit PV MMA
   static constexpr int PV_STEPS = BLK / PV_KEYS;
   static constexpr int NUM_BARS = 2 + 2 * (K_STAGES + V_STAGES + V8_STAGES) + 8 + 1 + 2 * kUnitRing;
@@ -371,10 +374,10 @@ __device__ __forceinline__ void load_pages(const AttnArgs& a, const Unit& U, Til
 
 // Copies of the K or V tile of a visited block whose pages were loaded raw:
 // out-of-range page ids are reported and read as zeros (outside the pool).
-template <bool FP8, int BLK, bool PAGED>
+template <bool FP8, int BLK, bool PAGED, int D>
 __device__ __forceinline__ void issue_kv_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, const AttnArgs& a,
                                               const Unit& U, const TileSrc<BLK>& t) {
-  using C = Cfg<FP8, BLK>;
+  using C = Cfg<FP8, BLK, D>;
   const Geometry& g = a.g;
   if constexpr (!PAGED) {
 #pragma unroll
@@ -400,11 +403,11 @@ __device__ __forceinline__ void issue_kv_tile(uint8_t* dst, const CUtensorMap* m
   }
 }
 
-template <bool FP8, int BLK, bool PAGED>
+template <bool FP8, int BLK, bool PAGED, int D>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
-  using C = Cfg<FP8, BLK>;
+  using C = Cfg<FP8, BLK, D>;
   constexpr int KS = C::K_STAGES, VS = C::V_STAGES, V8S = C::V8_STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -492,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      long long kt = 0, vt = 0, qn = 0;
+      int kt = 0, vt = 0, qn = 0;  // ring positions (tiles a CTA moves stay far below 2^31)
       const uint32_t q_bytes = 2u * C::DCH * a.rows * 128u;
       constexpr int VLS = FP8 ? V8S : VS;
       constexpr int VL_TILE = FP8 ? C::V8_TILE : C::V_TILE;
@@ -533,14 +536,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(k_empty + st, (uint32_t)((kt / KS) & 1) ^ 1u, abort_flag, g.status, FP_DEV_TIMEOUT);
           if (!ok) break;
           mbar_arrive_expect_tx(k_full + st, C::K_TILE);
-          issue_kv_tile<FP8, BLK, PAGED>(sK + st * C::K_TILE, &tmK, k_full + st, a, U, cur);
+          issue_kv_tile<FP8, BLK, PAGED, D>(sK + st * C::K_TILE, &tmK, k_full + st, a, U, cur);
           ++kt;
           // V: straight into the 16-bit ring (bf16) or into the e4m3 ring the converter reads
           st = (int)(vt % VLS);
           ok = mbar_wait(vl_empty + st, (uint32_t)((vt / VLS) & 1) ^ 1u, abort_flag, g.status, FP_DEV_TIMEOUT);
           if (!ok) break;
           mbar_arrive_expect_tx(vl_full + st, VL_TILE);
-          issue_kv_tile<FP8, BLK, PAGED>(sVL + st * VL_TILE, &tmV, vl_full + st, a, U, cur);
+          issue_kv_tile<FP8, BLK, PAGED, D>(sVL + st * VL_TILE, &tmV, vl_full + st, a, U, cur);
           ++vt;
           cur = nxt;
         }
@@ -548,9 +551,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Every copy this CTA issued lands before its shared memory is released,
       // also when another role gave up after this loop ended (on the normal
       // path the consumers have already seen these phases complete).
-      for (long long t = kt - 1; t >= 0 && t >= kt - KS; --t)
+      for (int t = kt - 1; t >= 0 && t >= kt - KS; --t)
         mbar_drain(k_full + (int)(t % KS), (uint32_t)((t / KS) & 1), g.status, FP_DEV_TIMEOUT);
-      for (long long t = vt - 1; t >= 0 && t >= vt - VLS; --t)
+      for (int t = vt - 1; t >= 0 && t >= vt - VLS; --t)
         mbar_drain(vl_full + (int)(t % VLS), (uint32_t)((t / VLS) & 1), g.status, FP_DEV_TIMEOUT);
       if (qn > 0) mbar_drain(q_full, (uint32_t)((qn - 1) & 1), g.status, FP_DEV_TIMEOUT);
     }
@@ -561,10 +564,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // PV: kind::f16, f16 (format 0) for e4m3 inputs or bf16 (format 1)
       const uint32_t fmt = FP8 ? 0u : 1u;
       const uint32_t idesc_qk = instr_desc(fmt, 128, BLK, 0, 0);
-      const uint32_t idesc_pv = instr_desc(fmt, 128, 128, 0, 1);
+      const uint32_t idesc_pv = instr_desc(fmt, 128, D, 0, 1);  // N = head dim
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-      long long kt = 0, vt = 0, qn = 0;
-      long long pn[2] = {0, 0};
+      int kt = 0, vt = 0, qn = 0;  // ring positions (tiles a CTA moves stay far below 2^31)
+      int pn[2] = {0, 0};
       bool ok = true;
 
       // Descriptors of the tiles' first bytes; an operand at byte offset `off`
@@ -673,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Widens every V tile the producer loads, in the same order, from the e4m3
     // ring into the f16 ring the PV MMAs read; exact (e4m3 is a subset of f16).
     const int ct = threadIdx.x - kConvertWarp * 32;  // 0..63
-    long long vt = 0;
+    int vt = 0;
     bool ok = true;
     UnitIter it{a.queue, a.order, unit_ring, unit_full, unit_empty, abort_flag, g.status, false, true, a.num_units, 0, 0};
     for (long long u = it.step(true, ok); u < a.num_units && ok; u = it.step(false, ok)) {
@@ -703,7 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + lane_base + mt * 128;
     const uint32_t tO = tmem + lane_base + 256 + mt * 128;
     const int hh = row % g.G, tt = row / g.G;
-    long long sn = 0, on = 0;
+    int sn = 0, on = 0;
     bool ok = true;
     UnitIter it{a.queue, a.order, unit_ring, unit_full, unit_empty, abort_flag, g.status, false, true, a.num_units, 0, 0};
     for (long long u = it.step(true, ok); u < a.num_units && ok; u = it.step(false, ok)) {
@@ -778,7 +781,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // TMEM accesses are warp-collective: rescale when any row of the warp needs it
         if (n > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < D / 16; ++c) {
             uint32_t r16[16];
             tmem_ld16(tO + c * 16, r16);
             tmem_wait_ld();
@@ -827,10 +830,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // epilogue: O / l -> bf16, natural-log LSE
-      __nv_bfloat16* orow_ptr = a.o + (orow * g.Hq + h) * 128;
+      __nv_bfloat16* orow_ptr = a.o + (orow * g.Hq + h) * D;
       if (U.count == 0) {
         if (valid) {
-          for (int c = 0; c < 16; ++c) reinterpret_cast<uint4*>(orow_ptr)[c] = make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow_ptr)[c] = make_uint4(0, 0, 0, 0);
           if (a.lse) a.lse[(long long)h * a.T + orow] = -INFINITY;
         }
         continue;
@@ -840,9 +843,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++on;
       tc_fence_after();
       const float inv = l > 0.f ? vmul / l : 0.f;  // a row that saw no key (masked everywhere) gets O = 0
-      // the O row in two TMEM round trips of 64 columns
+      // the O row in TMEM round trips of 64 columns
 #pragma unroll
-      for (int hc = 0; hc < 2; ++hc) {
+      for (int hc = 0; hc < D / 64; ++hc) {
         uint32_t r[64];
         tmem_ld32(tO + hc * 64, r);
         tmem_ld32(tO + hc * 64 + 32, r + 32);
@@ -889,33 +892,33 @@ int sm_count() {
   return n;
 }
 
-template <bool FP8, int BLK, bool PAGED>
+template <bool FP8, int BLK, bool PAGED, int D>
 fp_status_t run(const AttnArgs& a, const void* q, const void* k, const void* v, cudaStream_t s, bool pdl) {
-  using C = Cfg<FP8, BLK>;
+  using C = Cfg<FP8, BLK, D>;
   const Geometry& g = a.g;
   const cuuint64_t es = FP8 ? 1 : 2;
   CUtensorMap mq, mk, mv;
   {
-    const cuuint64_t dims[3] = {128, (cuuint64_t)g.Hq, (cuuint64_t)a.T};
-    const cuuint64_t strides[2] = {128 * es, (cuuint64_t)g.Hq * 128 * es};
+    const cuuint64_t dims[3] = {D, (cuuint64_t)g.Hq, (cuuint64_t)a.T};
+    const cuuint64_t strides[2] = {D * es, (cuuint64_t)g.Hq * D * es};
     const cuuint32_t box[3] = {(cuuint32_t)C::CH_ELEMS, (cuuint32_t)g.G, (cuuint32_t)a.Tm};
     if (!encode(&mq, FP8, 3, q, dims, strides, box)) return FP_ERR_CUDA;
   }
   if (!PAGED) {
-    const cuuint64_t dims[3] = {128, (cuuint64_t)g.Hkv, (cuuint64_t)a.T};
-    const cuuint64_t strides[2] = {128 * es, (cuuint64_t)g.Hkv * 128 * es};
+    const cuuint64_t dims[3] = {D, (cuuint64_t)g.Hkv, (cuuint64_t)a.T};
+    const cuuint64_t strides[2] = {D * es, (cuuint64_t)g.Hkv * D * es};
     const cuuint32_t box[3] = {(cuuint32_t)C::CH_ELEMS, 1, (cuuint32_t)BLK};
     if (!encode(&mk, FP8, 3, k, dims, strides, box) || !encode(&mv, FP8, 3, v, dims, strides, box))
       return FP_ERR_CUDA;
   } else {
     const cuuint64_t P = (cuuint64_t)g.page_size;
-    const cuuint64_t dims[4] = {128, (cuuint64_t)g.Hkv, P, (cuuint64_t)g.num_pages};
-    const cuuint64_t strides[3] = {128 * es, (cuuint64_t)g.Hkv * 128 * es, P * g.Hkv * 128 * es};
+    const cuuint64_t dims[4] = {D, (cuuint64_t)g.Hkv, P, (cuuint64_t)g.num_pages};
+    const cuuint64_t strides[3] = {D * es, (cuuint64_t)g.Hkv * D * es, P * g.Hkv * D * es};
     const cuuint32_t box[4] = {(cuuint32_t)C::CH_ELEMS, 1, (cuuint32_t)(g.page_size < BLK ? g.page_size : BLK), 1};
     if (!encode(&mk, FP8, 4, k, dims, strides, box) || !encode(&mv, FP8, 4, v, dims, strides, box))
       return FP_ERR_CUDA;
   }
-  auto kern = sparse_attention_kernel<FP8, BLK, PAGED>;
+  auto kern = sparse_attention_kernel<FP8, BLK, PAGED, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) {
     set_last_error("attention smem attribute", (int)e, cudaGetErrorString(e));
@@ -1054,13 +1057,21 @@ fp_status_t launch_attention(const Geometry& g, const void* q, const void* k, co
   a.o = reinterpret_cast<__nv_bfloat16*>(o);
   a.lse = lse;
   const bool paged = g.page_table != nullptr;
-  if (g.B == 128) {
-    if (g.fp8) return paged ? run<true, 128, true>(a, q, k, v, s, pdl) : run<true, 128, false>(a, q, k, v, s, pdl);
-    return paged ? run<false, 128, true>(a, q, k, v, s, pdl) : run<false, 128, false>(a, q, k, v, s, pdl);
+  if (g.d == 128) {
+    if (g.B == 128) {
+      if (g.fp8) return paged ? run<true, 128, true, 128>(a, q, k, v, s, pdl) : run<true, 128, false, 128>(a, q, k, v, s, pdl);
+      return paged ? run<false, 128, true, 128>(a, q, k, v, s, pdl) : run<false, 128, false, 128>(a, q, k, v, s, pdl);
+    }
+    if (g.B == 64) {
+      if (g.fp8) return paged ? run<true, 64, true, 128>(a, q, k, v, s, pdl) : run<true, 64, false, 128>(a, q, k, v, s, pdl);
+      return paged ? run<false, 64, true, 128>(a, q, k, v, s, pdl) : run<false, 64, false, 128>(a, q, k, v, s, pdl);
+    }
   }
-  if (g.B == 64) {
-    if (g.fp8) return paged ? run<true, 64, true>(a, q, k, v, s, pdl) : run<true, 64, false>(a, q, k, v, s, pdl);
-    return paged ? run<false, 64, true>(a, q, k, v, s, pdl) : run<false, 64, false>(a, q, k, v, s, pdl);
+  if (g.d == 64 && !g.fp8) {  // e4m3 rows of 64 bytes are not supported
+    if (g.B == 128)
+      return paged ? run<false, 128, true, 64>(a, q, k, v, s, pdl) : run<false, 128, false, 64>(a, q, k, v, s, pdl);
+    if (g.B == 64)
+      return paged ? run<false, 64, true, 64>(a, q, k, v, s, pdl) : run<false, 64, false, 64>(a, q, k, v, s, pdl);
   }
   return FP_ERR_UNSUPPORTED;
 }

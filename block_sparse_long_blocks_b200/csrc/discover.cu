@@ -88,9 +88,9 @@ __device__ __forceinline__ void split3(float x, uint16_t& h, uint16_t& m, uint16
 }
 
 // Grid: first the Q work items (request, block, head chunk), then the K ones.
-// Q items write the planes qpl[3][R * Nmax][Hq][128]; K items write
-// kpl[3][R * Hkv][Nmax][128] (both bf16, plane 0 = hi, 1 = mid, 2 = lo).
-template <bool FP8>
+// Q items write the planes qpl[3][R * Nmax][Hq][D]; K items write
+// kpl[3][R * Hkv][Nmax][D] (both bf16, plane 0 = hi, 1 = mid, 2 = lo).
+template <bool FP8, int D>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geometry g, const uint8_t* __restrict__ q,
                                                             const uint8_t* __restrict__ k,
                                                             __nv_bfloat16* __restrict__ qpl,
@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geometry g, const ui
                                                             int n_q_items) {
   constexpr int ES = FP8 ? 1 : 2;      // element size
   constexpr int EPV = 16 / ES;         // elements per 16-byte vector
-  constexpr int VPH = 128 / EPV;       // vectors per head row (d = 128)
+  constexpr int VPH = D / EPV;         // vectors per head row
   __shared__ __align__(16) float red[kPoolThreads * EPV];
 
   int item = blockIdx.x;
@@ -127,8 +127,8 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geometry g, const ui
   const int e0 = (v % VPH) * EPV;
   const uint8_t* base = isK ? k : q;
   const bool paged = isK && g.page_table != nullptr;
-  const long long head_off = ((long long)h * 128 + e0) * ES;
-  const long long row_bytes = (long long)H * 128 * ES;
+  const long long head_off = ((long long)h * D + e0) * ES;
+  const long long row_bytes = (long long)H * D * ES;
 
   float acc[EPV];
 #pragma unroll
@@ -199,9 +199,9 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geometry g, const ui
   uint16_t part[3][EPV];
 #pragma unroll
   for (int e = 0; e < EPV; ++e) split3(acc[e] * mul, part[0][e], part[1][e], part[2][e]);
-  const long long plane = isK ? (long long)g.R * g.Hkv * g.Nmax * 128 : (long long)g.R * g.Nmax * g.Hq * 128;
-  __nv_bfloat16* dst = isK ? kpl + (((long long)r * g.Hkv + h) * g.Nmax + i) * 128 + e0
-                           : qpl + (((long long)r * g.Nmax + i) * g.Hq + h) * 128 + e0;
+  const long long plane = isK ? (long long)g.R * g.Hkv * g.Nmax * D : (long long)g.R * g.Nmax * g.Hq * D;
+  __nv_bfloat16* dst = isK ? kpl + (((long long)r * g.Hkv + h) * g.Nmax + i) * D + e0
+                           : qpl + (((long long)r * g.Nmax + i) * g.Hq + h) * D + e0;
 #pragma unroll
   for (int pl = 0; pl < 3; ++pl) {
 #pragma unroll
@@ -225,7 +225,12 @@ constexpr int kScoreMmaWarp = 5;
 constexpr int kTile = 128 * 128;    // 128 rows x 64 bf16: one 128-byte swizzled row per score row / key block
 constexpr int kScoreStages = 2;     // key ring: one stage = the three planes of one 64-wide d chunk
 constexpr int kScoreBars = 1 + 2 * kScoreStages + 4 + 1;
-constexpr int kScoreSmem = 1024 + 6 * kTile + kScoreStages * 3 * kTile + 128 * 4 * 4 + 128 * 4 + kScoreBars * 8 + 64;
+// DC = D / 64 chunks of 64 pooled dimensions (one 128-byte swizzled row each)
+template <int DC>
+struct ScoreSmem {
+  static constexpr int value = 1024 + 3 * DC * kTile + kScoreStages * 3 * kTile + 128 * 4 * 4 + 128 * 4 +
+                               kScoreBars * 8 + 64;
+};
 // plane pairs of the six products, largest terms first
 __constant__ int8_t kProdA[6] = {0, 0, 1, 1, 0, 2};
 __constant__ int8_t kProdB[6] = {0, 1, 0, 1, 2, 0};
@@ -252,7 +257,7 @@ __device__ __forceinline__ uint32_t bit_range(int jb, int lo, int hi) {
   return upto & ~((1u << a) - 1u);
 }
 
-template <int G>
+template <int G, int DC>
 __global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK, const Geometry g,
                  uint32_t a_bytes, uint32_t b_bytes, uint32_t* __restrict__ mask, int32_t* __restrict__ idx,
@@ -262,7 +267,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;                                   // [plane][d chunk] pooled queries
-  uint8_t* sB = sA + 6 * kTile;                         // [stage][plane] pooled keys
+  uint8_t* sB = sA + 3 * DC * kTile;                    // [stage][plane] pooled keys
   uint32_t* kw = reinterpret_cast<uint32_t*>(sB + kScoreStages * 3 * kTile);  // [row][4] keep words
   int* cbase = reinterpret_cast<int*>(kw + 128 * 4);  // [QB] list length so far
   uint64_t* bars = reinterpret_cast<uint64_t*>(cbase + 128);
@@ -329,15 +334,15 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
-      mbar_arrive_expect_tx(a_full, 6u * a_bytes);
+      mbar_arrive_expect_tx(a_full, 3u * DC * a_bytes);
       for (int pl = 0; pl < 3; ++pl)
-        for (int c = 0; c < 2; ++c)
-          tma_load_4d(sA + (pl * 2 + c) * kTile, &tmQ, a_full, c * 64, kvh * G, r * g.Nmax + i0, pl);
+        for (int c = 0; c < DC; ++c)
+          tma_load_4d(sA + (pl * DC + c) * kTile, &tmQ, a_full, c * 64, kvh * G, r * g.Nmax + i0, pl);
       bool ok = true;
       int n = 0;
       for (int pass = 0; pass < 2 && ok; ++pass)
         for (int nt = 0; nt < NT && ok; ++nt)
-          for (int c = 0; c < 2; ++c, ++n) {
+          for (int c = 0; c < DC; ++c, ++n) {
             const int st = n % kScoreStages;
             ok = mbar_wait(b_empty + st, (uint32_t)((n / kScoreStages) & 1) ^ 1u, abort_flag, g.status,
                            FP_DEV_TIMEOUT);
@@ -366,7 +371,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
           ok = mbar_wait(s_empty + buf, (uint32_t)((q >> 1) & 1) ^ 1u, abort_flag, g.status, FP_DEV_TIMEOUT);
           if (!ok) break;
           tc_fence_after();
-          for (int c = 0; c < 2 && ok; ++c, ++n) {
+          for (int c = 0; c < DC && ok; ++c, ++n) {
             const int st = n % kScoreStages;
             ok = mbar_wait(b_full + st, (uint32_t)((n / kScoreStages) & 1), abort_flag, g.status, FP_DEV_TIMEOUT);
             if (!ok) break;
@@ -375,7 +380,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             for (int ks = 0; ks < 4; ++ks) {
 #pragma unroll
               for (int pr = 0; pr < 6; ++pr) {
-                const uint64_t ad = smem_desc_sw128(sAa + (kProdA[pr] * 2 + c) * kTile + ks * 32, 16, 1024);
+                const uint64_t ad = smem_desc_sw128(sAa + (kProdA[pr] * DC + c) * kTile + ks * 32, 16, 1024);
                 const uint64_t bd = smem_desc_sw128(sBa + (st * 3 + kProdB[pr]) * kTile + ks * 32, 16, 1024);
                 umma_f16_ss(tmem + buf * 128, ad, bd, idesc, (c | ks | pr) ? 1u : 0u);
               }
@@ -556,34 +561,37 @@ int pow2_divisor(int H, int cap) {
   return hc;
 }
 
-template <int G>
+template <int G, int DC>
 fp_status_t launch_score_g(const Geometry& g, const __nv_bfloat16* qpl, const __nv_bfloat16* kpl, uint32_t* mask,
                            int32_t* idx, int32_t* cnt, cudaStream_t s) {
   constexpr int QB = 128 / G;
-  // pooled queries: [3][R * Nmax][Hq][128], box = one 64-wide d chunk of G heads x QB blocks
+  // pooled queries: [3][R * Nmax][Hq][D], box = one 64-wide d chunk of G heads x QB blocks
   const int qb_box = QB < g.R * g.Nmax ? QB : g.R * g.Nmax;
   const int kb_box = g.Nmax < 128 ? g.Nmax : 128;
   CUtensorMap mq, mk;
   {
-    const cuuint64_t dims[4] = {128, (cuuint64_t)g.Hq, (cuuint64_t)g.R * g.Nmax, 3};
-    const cuuint64_t strides[3] = {256, (cuuint64_t)g.Hq * 256, (cuuint64_t)g.R * g.Nmax * g.Hq * 256};
+    const cuuint64_t row = 2 * 64 * DC;  // bytes of one pooled bf16 row
+    const cuuint64_t dims[4] = {64 * DC, (cuuint64_t)g.Hq, (cuuint64_t)g.R * g.Nmax, 3};
+    const cuuint64_t strides[3] = {row, (cuuint64_t)g.Hq * row, (cuuint64_t)g.R * g.Nmax * g.Hq * row};
     const cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)qb_box, 1};
     if (!encode_tiled(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, qpl, dims, strides, box)) return FP_ERR_CUDA;
   }
   {
-    const cuuint64_t dims[4] = {128, (cuuint64_t)g.Nmax, (cuuint64_t)g.R * g.Hkv, 3};
-    const cuuint64_t strides[3] = {256, (cuuint64_t)g.Nmax * 256, (cuuint64_t)g.R * g.Hkv * g.Nmax * 256};
+    const cuuint64_t row = 2 * 64 * DC;
+    const cuuint64_t dims[4] = {64 * DC, (cuuint64_t)g.Nmax, (cuuint64_t)g.R * g.Hkv, 3};
+    const cuuint64_t strides[3] = {row, (cuuint64_t)g.Nmax * row, (cuuint64_t)g.R * g.Hkv * g.Nmax * row};
     const cuuint32_t box[4] = {64, (cuuint32_t)kb_box, 1, 1};
     if (!encode_tiled(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, kpl, dims, strides, box)) return FP_ERR_CUDA;
   }
-  cudaError_t e = cudaFuncSetAttribute(score_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kScoreSmem);
+  constexpr int kSmem = ScoreSmem<DC>::value;
+  cudaError_t e = cudaFuncSetAttribute(score_kernel<G, DC>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) {
     set_last_error("score smem attribute", (int)e, cudaGetErrorString(e));
     return FP_ERR_CUDA;
   }
   const unsigned grid = (unsigned)(g.R * g.Hkv * ((g.Nmax + QB - 1) / QB));
   const uint32_t a_bytes = 128u * G * qb_box, b_bytes = 128u * kb_box;
-  score_kernel<G><<<grid, kScoreThreads, kScoreSmem, s>>>(mq, mk, g, a_bytes, b_bytes, mask, idx, cnt);
+  score_kernel<G, DC><<<grid, kScoreThreads, kSmem, s>>>(mq, mk, g, a_bytes, b_bytes, mask, idx, cnt);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_last_error("score launch", (int)e, cudaGetErrorString(e));
@@ -594,8 +602,8 @@ fp_status_t launch_score_g(const Geometry& g, const __nv_bfloat16* qpl, const __
 
 }  // namespace
 
-size_t pooled_q_elems(const Geometry& g) { return (size_t)g.R * g.Nmax * g.Hq * 128; }
-size_t pooled_k_elems(const Geometry& g) { return (size_t)g.R * g.Hkv * g.Nmax * 128; }
+size_t pooled_q_elems(const Geometry& g) { return (size_t)g.R * g.Nmax * g.Hq * g.d; }
+size_t pooled_k_elems(const Geometry& g) { return (size_t)g.R * g.Hkv * g.Nmax * g.d; }
 
 cudaError_t launch_pool(const Geometry& g, const void* q, const void* k, __nv_bfloat16* qpl, __nv_bfloat16* kpl,
                         cudaStream_t s) {
@@ -603,27 +611,38 @@ cudaError_t launch_pool(const Geometry& g, const void* q, const void* k, __nv_bf
   const int hcq = pow2_divisor(g.Hq, cap), hck = pow2_divisor(g.Hkv, cap);
   const int nq = g.R * g.Nmax * (g.Hq / hcq);
   const int nk = g.R * g.Nmax * (g.Hkv / hck);
-  if (g.fp8)
-    pool_kernel<true><<<nq + nk, kPoolThreads, 0, s>>>(g, (const uint8_t*)q, (const uint8_t*)k, qpl, kpl, hcq, hck,
-                                                       nq);
+  const uint8_t *q8 = (const uint8_t*)q, *k8 = (const uint8_t*)k;
+  if (g.fp8)  // e4m3 inputs: head dim 128
+    pool_kernel<true, 128><<<nq + nk, kPoolThreads, 0, s>>>(g, q8, k8, qpl, kpl, hcq, hck, nq);
+  else if (g.d == 128)
+    pool_kernel<false, 128><<<nq + nk, kPoolThreads, 0, s>>>(g, q8, k8, qpl, kpl, hcq, hck, nq);
   else
-    pool_kernel<false><<<nq + nk, kPoolThreads, 0, s>>>(g, (const uint8_t*)q, (const uint8_t*)k, qpl, kpl, hcq,
-                                                        hck, nq);
+    pool_kernel<false, 64><<<nq + nk, kPoolThreads, 0, s>>>(g, q8, k8, qpl, kpl, hcq, hck, nq);
   return cudaGetLastError();
 }
 
 fp_status_t launch_score(const Geometry& g, const __nv_bfloat16* qpl, const __nv_bfloat16* kpl, uint32_t* mask,
                          int32_t* idx, int32_t* cnt, cudaStream_t s) {
+  const bool dc2 = g.d == 128;  // pooled rows of 128 (two 64-wide chunks) or 64 dimensions
   switch (g.G) {
-    case 1: return launch_score_g<1>(g, qpl, kpl, mask, idx, cnt, s);
-    case 2: return launch_score_g<2>(g, qpl, kpl, mask, idx, cnt, s);
-    case 3: return launch_score_g<3>(g, qpl, kpl, mask, idx, cnt, s);
-    case 4: return launch_score_g<4>(g, qpl, kpl, mask, idx, cnt, s);
-    case 5: return launch_score_g<5>(g, qpl, kpl, mask, idx, cnt, s);
-    case 6: return launch_score_g<6>(g, qpl, kpl, mask, idx, cnt, s);
-    case 7: return launch_score_g<7>(g, qpl, kpl, mask, idx, cnt, s);
-    case 8: return launch_score_g<8>(g, qpl, kpl, mask, idx, cnt, s);
-    case 16: return launch_score_g<16>(g, qpl, kpl, mask, idx, cnt, s);
+    case 1: return dc2 ? launch_score_g<1, 2>(g, qpl, kpl, mask, idx, cnt, s)
+                  : launch_score_g<1, 1>(g, qpl, kpl, mask, idx, cnt, s);
+    case 2: return dc2 ? launch_score_g<2, 2>(g, qpl, kpl, mask, idx, cnt, s)
+                  : launch_score_g<2, 1>(g, qpl, kpl, mask, idx, cnt, s);
+    case 3: return dc2 ? launch_score_g<3, 2>(g, qpl, kpl, mask, idx, cnt, s)
+                  : launch_score_g<3, 1>(g, qpl, kpl, mask, idx, cnt, s);
+    case 4: return dc2 ? launch_score_g<4, 2>(g, qpl, kpl, mask, idx, cnt, s)
+                  : launch_score_g<4, 1>(g, qpl, kpl, mask, idx, cnt, s);
+    case 5: return dc2 ? launch_score_g<5, 2>(g, qpl, kpl, mask, idx, cnt, s)
+                  : launch_score_g<5, 1>(g, qpl, kpl, mask, idx, cnt, s);
+    case 6: return dc2 ? launch_score_g<6, 2>(g, qpl, kpl, mask, idx, cnt, s)
+                  : launch_score_g<6, 1>(g, qpl, kpl, mask, idx, cnt, s);
+    case 7: return dc2 ? launch_score_g<7, 2>(g, qpl, kpl, mask, idx, cnt, s)
+                  : launch_score_g<7, 1>(g, qpl, kpl, mask, idx, cnt, s);
+    case 8: return dc2 ? launch_score_g<8, 2>(g, qpl, kpl, mask, idx, cnt, s)
+                  : launch_score_g<8, 1>(g, qpl, kpl, mask, idx, cnt, s);
+    case 16: return dc2 ? launch_score_g<16, 2>(g, qpl, kpl, mask, idx, cnt, s)
+                  : launch_score_g<16, 1>(g, qpl, kpl, mask, idx, cnt, s);
     default: return FP_ERR_UNSUPPORTED;
   }
 }

@@ -82,7 +82,7 @@ extern "C" {
 typedef enum {
   FP_OK = 0,
   FP_ERR_INVALID_ARG = -1,  /* null pointer, bad size, alpha < 0 or not finite */
-  FP_ERR_UNSUPPORTED = -2,  /* head_dim != 128, block not 64/128, G = hq / hkv not in
+  FP_ERR_UNSUPPORTED = -2,  /* head_dim not 128 (or 64 with bf16), block not 64/128, G = hq / hkv not in
                                1..8 or 16, Nmax > 8192, page size not a power of two in
                                16..65536 */
   FP_ERR_ALIGNMENT = -3,    /* a tensor pointer is not 16-byte aligned */
@@ -104,7 +104,7 @@ typedef struct {
   int batch;               /* contiguous layout: number of sequences; varlen: number of requests R */
   int max_seqlen;          /* contiguous: tokens per sequence; varlen: upper bound on every length */
   int hq, hkv;             /* query heads, KV heads; hq % hkv == 0 */
-  int head_dim;            /* must be 128 */
+  int head_dim;            /* 128, or 64 with bf16 inputs */
   int block;               /* B: 64 or 128 tokens */
   float alpha;             /* dynamic-threshold factor, finite and >= 0 */
   int sink_tokens;         /* leading tokens always kept: ceil(sink_tokens / B) blocks */
@@ -217,11 +217,16 @@ fp_status_t fp_prefill(const fp_params_t* p, const void* q, const void* k, const
  * - Limit: fp_workspace_size(p) must not exceed fp_static_scratch_bytes()
  *   (32 MiB, enough for one 128K-token sequence with 32 query / 4 KV heads at
  *   block 128); larger problems return FP_ERR_WORKSPACE before any launch and
- *   fp_last_error() says how much was needed.
+ *   fp_last_error() says how much was needed. The limit is checked against
+ *   the whole fp_workspace_size, which also counts the attention's queue
+ *   area that discovery does not use, so it errs on the safe side.
  * - The array exists on every GPU that loads the library, until exit. The
  *   first call on a device looks up the array's device address on that
- *   device (the device must be current); make that first call before any
- *   stream capture.
+ *   device (the device must be current) and keeps it for the life of the
+ *   process; make that first call before any stream capture. A
+ *   cudaDeviceReset() of that device invalidates the kept address: calling
+ *   this entry point (or fp_get_device_status, which keeps the status word's
+ *   address the same way) on a device after resetting it is not supported.
  * - All calls share the one array and it keeps the last call's contents
  *   (nothing in it needs to start at zero). Calls whose work overlaps on the
  *   GPU (e.g. on two streams at once) race on it: serialise them.

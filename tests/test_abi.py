@@ -61,17 +61,18 @@ def _pad256(n):
 
 @pytest.mark.parametrize("kw,pairs", [({}, 4), (dict(hq=4), 1), (dict(hkv=2), 8), (dict(hq=6, hkv=2), 2)])
 def test_workspace_layout(lib, kw, pairs):
-    """Pooled query and key planes (three bf16 parts each), the work-queue
-    counter and the claim order of the attention's work units: M-tile pairs
-    per query block = B / (2 Tm), Tm the largest power of two with Tm G <= 128
-    and Tm <= B / 2."""
-    cfg = _cfg(**kw)
-    p = fb.make_params(cfg)
-    N, R, Hq, Hkv = cfg.nmax, cfg.batch, cfg.hq, cfg.hkv
-    q_planes = _pad256(3 * 2 * R * N * Hq * 128)
-    k_planes = _pad256(3 * 2 * R * Hkv * N * 128)
-    order = _pad256(4 * N * R * Hkv * pairs)
-    assert fb.sizes(p)["workspace"] == q_planes + k_planes + 256 + order
+    """Pooled query and key planes (three bf16 parts each, d values per row),
+    the work-queue counter and the claim order of the attention's work units:
+    M-tile pairs per query block = B / (2 Tm), Tm the largest power of two with
+    Tm G <= 128 and Tm <= B / 2."""
+    for d in (128, 64):
+        cfg = _cfg(head_dim=d, **kw)
+        p = fb.make_params(cfg)
+        N, R, Hq, Hkv = cfg.nmax, cfg.batch, cfg.hq, cfg.hkv
+        q_planes = _pad256(3 * 2 * R * N * Hq * d)
+        k_planes = _pad256(3 * 2 * R * Hkv * N * d)
+        order = _pad256(4 * N * R * Hkv * pairs)
+        assert fb.sizes(p)["workspace"] == q_planes + k_planes + 256 + order
 
 
 def test_single_call_argument_checks(lib):
@@ -87,7 +88,7 @@ def test_single_call_argument_checks(lib):
 
 
 @pytest.mark.parametrize("bad,code", [
-    (dict(head_dim=64), -2), (dict(block=32), -2), (dict(alpha=-0.5), -1), (dict(alpha=float("nan")), -1),
+    (dict(head_dim=96), -2), (dict(head_dim=256), -2), (dict(head_dim=64, fp8=True), -2), (dict(block=32), -2), (dict(alpha=-0.5), -1), (dict(alpha=float("nan")), -1),
     (dict(alpha=float("inf")), -1), (dict(hq=30, hkv=4), -1), (dict(batch=0), -1), (dict(max_seqlen=0), -1),
     (dict(sink_tokens=-1), -1), (dict(hq=36, hkv=4), -2), (dict(max_seqlen=128 * 8193), -2),
 ])

@@ -19,14 +19,16 @@ from block_sparse_long_blocks_b200 import workloads as wl
 
 @pytest.mark.gpu
 def test_static_scratch_matches_workspace_entry_on_consecutive_calls():
-    fb.load()
+    lib = fb.load()
     cases = [wl.small_case(wl.workloads()["qwen30b_128k"], 8192),
              wl.workloads()["tiny2k"],
-             wl.small_case(wl.workloads()["extreme_256k"], 5000)]
+             wl.small_case(wl.workloads()["extreme_256k"], 5000),
+             wl.workloads()["qwen30b_128k"]]  # the full 128K sequence the size limit is stated for
     for w in cases:
         inp = wl.make_inputs(w)
         cfg = fb.config_for(w, inp)
         p = fb.make_params(cfg)
+        assert lib.fp_workspace_size(ctypes.byref(p)) <= lib.fp_static_scratch_bytes()
         q, k = inp.q.cuda(), inp.k.cuda()
         ref = fb.Buffers(p)
         fb.fp_discover_compact(p, q, k, ref.mask, ref.idx, ref.cnt, ref.workspace)
